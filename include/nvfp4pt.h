@@ -1,0 +1,165 @@
+/*
+ * nvfp4pt.h -- C ABI of the B200 (sm_100a) NVFP4 per-token quantization cast.
+ *
+ * The cast (TransformerEngine PR #3045 "Add NVFP4 per-token quantization recipe",
+ * Description): where the default NVFP4 recipe keeps one outer amax per tensor,
+ * the per-token recipe keeps one per row (length M) for the rowwise data and one
+ * per column (length K) for the columnwise data. With
+ *     s_enc = 2688 / amax        (binary32, round-to-nearest-even; 1 when amax == 0)
+ * each 16-element block gets an E4M3 scale
+ *     sf    = e4m3_rn_satfinite( RN( RN(block_amax / 6) * s_enc ) )
+ * (the order of the weight quantizer's (amax/6) * 448 / (gA/6), Model-Optimizer
+ * PR #2598, review thread on the FP8 block scale: other orders round to other codes),
+ *     enc   = sf == 0 ? 0 : RN(s_enc / float(sf))
+ * and each element becomes q = e2m1_rn_satfinite(RN(x * enc)), two codes per byte,
+ * element 2j in the low nibble. Readings where the pages are silent: s_enc and enc
+ * are clamped to FLT_MAX instead of overflowing; a negative value that rounds to
+ * zero keeps its sign (code 0x8); NaN/inf inputs are outside the contract.
+ *
+ * Layouts ("compact" = unswizzled, TransformerEngine PR #3244, review):
+ *   x         bf16 row-major [rows, cols], leading dimension = cols.
+ *   q_row     uint8 [rows, cols/2]      codes of row r, block b at bytes 8b..8b+7.
+ *   sf_row    uint8 [rows, cols/16]     E4M3 scale of each 16-element row block.
+ *   amax_row  fp32  [rows]
+ *   q_col     uint8 [cols, rows/2]      the rowwise cast of x^T ("stored transposed").
+ *   sf_col    uint8 [cols, rows/16]
+ *   amax_col  fp32  [cols]              (grouped: [num_groups, cols])
+ *
+ * Conventions shared by every call:
+ *   - All array pointers are device pointers owned by the caller; the library keeps
+ *     no pointer after the call returns and allocates no device memory.
+ *   - Calls are asynchronous: the work is ordered on `stream` (0 = legacy default
+ *     stream), and outputs are valid once the stream reaches that point.
+ *   - rows and cols are > 0, multiples of 16, and at most 2^30; each pointer that is
+ *     used is non-NULL and 16-byte aligned. Violations are reported by the return
+ *     value BEFORE anything is launched; nothing is written then.
+ *   - A launch or CUDA API failure returns NVFP4PT_ERR_CUDA.
+ *   - Calls on one stream may reuse the same workspace; concurrent calls on
+ *     different streams need different workspaces.
+ *   - The library is for sm_100 (B200) devices only (NVFP4 is a Blackwell format;
+ *     PR #3045 gates its path to SM100 the same way): NVFP4PT_ERR_ARCH elsewhere.
+ */
+#ifndef NVFP4PT_H
+#define NVFP4PT_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4PT_OK = 0,
+    NVFP4PT_ERR_NULL = 1,      /* a pointer that the flags require is NULL              */
+    NVFP4PT_ERR_SHAPE = 2,     /* rows/cols not in (0, 2^30] or not multiples of 16      */
+    NVFP4PT_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned                      */
+    NVFP4PT_ERR_GROUPS = 4,    /* num_groups outside [1, 1024], or offsets not 0 = o[0] <=
+                                  o[1] <= ... <= o[G] = rows with every o[g] % 16 == 0   */
+    NVFP4PT_ERR_ARCH = 5,      /* the current device is not compute capability 10.0     */
+    NVFP4PT_ERR_CUDA = 6,      /* a CUDA call or a kernel launch failed                 */
+    NVFP4PT_ERR_FLAGS = 7,     /* flags is not a non-empty subset of ROWWISE|COLWISE    */
+    NVFP4PT_ERR_DEVICE = 8     /* a kernel reported a device-side error (see below)     */
+} nvfp4pt_status;
+
+/* Output selection. The same meaning, and the same default in the bindings
+ * (both directions), in every call: PR #3045's review found split APIs whose
+ * columnwise defaults disagreed. */
+enum { NVFP4PT_ROWWISE = 1, NVFP4PT_COLWISE = 2 };
+
+/* Maximum number of token groups of nvfp4pt_quantize_grouped. */
+#define NVFP4PT_MAX_GROUPS 1024
+
+/* A constant, human-readable name of a status code. Never NULL. */
+const char* nvfp4pt_status_string(nvfp4pt_status status);
+
+/* Bytes of device workspace a call with these sizes needs (num_groups = 1 for the
+ * ungrouped and weight calls). The workspace holds per-call scratch (the observed
+ * maxima of the absmax update and a device error word); it needs no initialisation
+ * and its contents after a call are unspecified except for the error word. */
+size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
+
+/*
+ * nvfp4pt_quantize -- per-token cast of x[rows, cols] (PR #3045, Description and
+ * Changes; the composite "vector amax, then encode" of its sequence diagram).
+ *
+ * flags      NVFP4PT_ROWWISE and/or NVFP4PT_COLWISE.
+ * q_row, sf_row, amax_row   rowwise outputs (required iff ROWWISE, else ignored).
+ * q_col, sf_col, amax_col   columnwise outputs (required iff COLWISE, else ignored).
+ * absmax_buf NULL, or one fp32 running buffer, updated in place with
+ *            New = max(RN(Old * decay), Observed), Observed = max |x| = max(amax_row)
+ *            (TransformerEngine PR #3296 "[PTQ] Store FP32 global scaling factors",
+ *            Description: decay 0 keeps the latest value, decay 1 the all-time max;
+ *            with per-token scales the row amaxes are max-reduced to a scalar).
+ * workspace  nvfp4pt_workspace_bytes(rows, cols, 1) bytes of device memory.
+ */
+nvfp4pt_status nvfp4pt_quantize(const void* x_bf16, int64_t rows, int64_t cols, int flags,
+                                uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                float* absmax_buf, float decay,
+                                void* workspace, cudaStream_t stream);
+
+/*
+ * nvfp4pt_quantize_grouped -- the cast of MoE token groups in one pass each
+ * (PR #3045, Important Files: the grouped per-token quantize helper that splits
+ * tokens per expert; its per-group metadata goes up in one batch). Group g is the
+ * row range [offsets_host[g], offsets_host[g+1]); empty groups are allowed (the
+ * page's helper rejects them; unbalanced routing produces them).
+ *
+ * offsets_host  HOST array of num_groups+1 row offsets (read during the call only).
+ * Rowwise outputs and amax_row are exactly those of nvfp4pt_quantize.
+ * amax_col   fp32 [num_groups, cols]: column amax over the group's rows (0 for an
+ *            empty group).
+ * q_col      group g's codes are [cols, m_g/2] starting at byte cols*offsets[g]/2.
+ * sf_col     group g's scales are [cols, m_g/16] starting at byte cols*offsets[g]/16.
+ * absmax_bufs NULL, or fp32 [num_groups]: one running buffer per group (one per
+ *            grouped GEMM, PR #3296 Important Files), Observed = max over the group's
+ *            rows (0 for an empty group, which then only decays).
+ * workspace  nvfp4pt_workspace_bytes(rows, cols, num_groups) bytes.
+ */
+nvfp4pt_status nvfp4pt_quantize_grouped(const void* x_bf16, int64_t rows, int64_t cols,
+                                        const int64_t* offsets_host, int num_groups, int flags,
+                                        uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                        uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                        float* absmax_bufs, float decay,
+                                        void* workspace, cudaStream_t stream);
+
+/*
+ * nvfp4pt_quantize_weight_2d -- the opt-in 2D weight cast (PR #3045, Changes:
+ * "transposition-invariant 16x16 cast emitted in per-token layout").
+ * Each row keeps its own s_enc from amax_row; the 16 rows of a band share one E4M3
+ * scale per 16-column block, sf = e4m3(max over the band's rows of
+ * RN(RN(block_amax/6) * s_enc[row])), which equals the largest of the 16 rowwise
+ * 1D scales; each row encodes with enc = RN(s_enc[row] / float(sf)). The shared
+ * scale is written to all 16 rows of the band: sf_row is [rows, cols/16] as in the
+ * 1D cast. Weights are kept rowwise only (PR #3296, Description).
+ * workspace  nvfp4pt_workspace_bytes(rows, cols, 1) bytes.
+ */
+nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w_bf16, int64_t rows, int64_t cols,
+                                          uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                          void* workspace, cudaStream_t stream);
+
+/*
+ * nvfp4pt_update_absmax -- the running-buffer step alone (PR #3296, Description):
+ * *absmax_buf = max(RN(*absmax_buf * decay), max_i amax_vec[i]); n may be 0
+ * (Observed = 0). Both pointers are device pointers; amax_vec holds n non-negative
+ * fp32 values. No workspace; n <= 2^40.
+ */
+nvfp4pt_status nvfp4pt_update_absmax(float* absmax_buf, const float* amax_vec, int64_t n,
+                                     float decay, cudaStream_t stream);
+
+/*
+ * nvfp4pt_workspace_error -- read the device error word the last call on this
+ * workspace left (0 = none). Synchronises `stream`. A nonzero word means a kernel
+ * gave up a bounded wait (a TMA copy that never arrived) and skipped the rest of its
+ * work; outputs of that call are then incomplete. Returns NVFP4PT_ERR_DEVICE if the
+ * word is nonzero, NVFP4PT_OK otherwise (the word is stored in *word if non-NULL).
+ */
+nvfp4pt_status nvfp4pt_workspace_error(const void* workspace, uint32_t* word, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4PT_H */
