@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 per-token cast on B200.
+
+One step = one call of nvfp4pt_quantize (zero -> fused row/column amax pass ->
+TMA encode pass, with the decayed running-absmax update) over the LLM-sized
+activation: bf16 [16384, 8192], N(0,1) with 1% outlier channels x50 (seed 2),
+rowwise + columnwise outputs, decay 0.99.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Each rank (one per GPU, torchrun for N > 1) casts its own independent matrix
+(replicas: the cast has no exchange step at this scale), so the work per GPU is
+fixed as N grows ("weak" scaling). Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain single-threaded C definition)
+on bounded row slices of the same matrix: the slow reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K = 16384, 8192
+DECAY = 0.99
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algo_bytes(m: int, k: int) -> int:
+    """Compulsory bytes of one cast: bf16 read twice, row and column codes and scales
+    written once, amax vectors written once."""
+    return 2 * (2 * m * k) + 2 * (m * k // 2) + 2 * (m * k // 16) + 4 * m + 4 * k
+
+
+def workload_name(m: int, k: int) -> str:
+    return f"llm_activation_{m}x{k}_bf16_rowcol_decay0.99"
+PROFILE_JSON = os.path.join(ROOT, "profiles", "nvfp4pt_cast_llm_16384x8192.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "precision_quantization_row_b200", "csrc", f)
+                  for f in ("nvfp4pt_api.cu", "nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh")]
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic():
+    """DRAM bytes per cast from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    try:
+        with open(PROFILE_JSON) as f:
+            d = json.load(f)
+        if d.get("kernel_source_sha") == kernel_source_sha():
+            return d.get("dram_bytes_per_cast")
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------- distributed
+
+class Dist:
+    """Rank bookkeeping. N = 1 runs without a process group."""
+
+    def __init__(self, gpus: int, backend: str | None = None):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != gpus:
+            raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={self.world}")
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            backend = backend or "nccl"
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            if self.pg.get_backend() == "nccl":
+                import torch
+                self.pg.barrier(device_ids=[torch.cuda.current_device()])
+            else:
+                self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        import torch
+        dev = "cuda" if self.pg.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def timed_region(dist: Dist, run, sync) -> float:
+    """Barrier + sync on both sides of `run`; returns the max over ranks of the
+    seconds `run` reports (device time)."""
+    dist.barrier()
+    sync()
+    secs = run()
+    sync()
+    dist.barrier()
+    return dist.max(secs)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+    REASONS = {  # NVML clocks-event reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return
+        self.period = period
+        self._t = threading.Thread(target=self._loop, daemon=True)
+
+    def _loop(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- GPU arm
+
+def run_gpu(args, dist: Dist) -> dict | None:
+    global M, K
+    M, K = args.rows, args.cols
+    import torch
+
+    import precision_quantization_row_b200 as nv
+    from precision_quantization_row_b200 import build, inputs
+
+    build.build()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    stream = torch.cuda.current_stream(dev)
+
+    x_host = inputs.llm(M=M, K=K)  # same matrix on every rank: independent replicas
+    # two input copies and two output sets, rotated every step (all > L2 in total)
+    xs = [x_host.to(dev), x_host.to(dev).clone()]
+    outs = [nv._outputs(M, K, nv.ROWWISE | nv.COLWISE, dev) for _ in range(2)]
+    buf = torch.zeros(1, dtype=torch.float32, device=dev)
+    ws = nv.new_workspace(M, K, device=dev)
+
+    def step(i):
+        nv.quantize(xs[i & 1], absmax=buf, decay=DECAY, out=outs[i & 1], workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if nv.workspace_error(ws) != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run():
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1) / 1e3
+
+    with ClockSampler(dev.index) as clk:
+        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    launches = 3 * args.steps  # zero, amax pass, encode pass per cast
+
+    # end to end through the public call with host buffers: pinned H2D of the input,
+    # the cast, D2H of every output (codes, scales, amax vectors, buffer)
+    e2e = None
+    if not args.no_e2e:
+        xh = x_host.pin_memory()
+        host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs[0].items()}
+        buf_h = torch.empty(1, dtype=torch.float32, pin_memory=True)
+        h2d = xh.numel() * xh.element_size()
+        d2h = sum(v.numel() * v.element_size() for v in host_out.values()) + buf_h.numel() * 4
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step(i):
+            xs[0].copy_(xh, non_blocking=True)
+            nv.quantize(xs[0], absmax=buf, decay=DECAY, out=outs[0], workspace=ws, stream=stream)
+            for k, v in outs[0].items():
+                host_out[k].copy_(v, non_blocking=True)
+            buf_h.copy_(buf, non_blocking=True)
+
+        for i in range(2):
+            e2e_step(i)
+
+        def run_e2e():
+            ev0.record(stream)
+            for i in range(e2e_steps):
+                e2e_step(i)
+            ev1.record(stream)
+            ev1.synchronize()
+            return ev0.elapsed_time(ev1) / 1e3
+
+        e2e_secs = timed_region(dist, run_e2e, lambda: torch.cuda.synchronize(dev))
+        e2e = {"value": float(M) * K * e2e_steps * dist.world / e2e_secs, "unit": "elem/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if nv.workspace_error(ws) != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    if dist.rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    per_cast = secs / args.steps
+    achieved = algo_bytes(M, K) / per_cast / 1e9
+    elems = float(M) * K
+    line = {
+        "metric": "NVFP4 per-token cast: elems/s, achieved HBM GB/s, % of B200 HBM peak",
+        "value": elems * args.steps * dist.world / secs,
+        "unit": "elem/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": per_cast * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16->nvfp4 (e2m1 codes, e4m3 scales, fp32 amax)",
+        "data": "synthetic",
+        "config": {"workload": workload_name(M, K), "rows": M, "cols": K, "flags": "rowwise+columnwise",
+                   "absmax_decay": DECAY, "parallelism": f"replicas x{dist.world}",
+                   "l2": f"inputs larger than L2 ({M * K * 2 / 1e6:.0f} MB each), 2 rotating input copies "
+                         "and output sets"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": ncu_traffic(), "peak_source": peak_kind,
+                     "nominal_frac_8TBs": achieved / 8000.0,
+                     "algorithmic_bytes_per_cast": algo_bytes(M, K)},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+# ------------------------------------------------------------ oracle arm
+
+def oracle_sample_rate(rows: int) -> tuple[float, str]:
+    """elems/s of the oracle's full row+col cast (with the absmax update) of the
+    first `rows` rows of the benchmark matrix, single-threaded."""
+    import oracle
+    from precision_quantization_row_b200 import inputs
+    x = inputs.llm()[:rows].contiguous()
+    xb = oracle._bits(x)
+    t = time.perf_counter()
+    oracle.quantize(xb, absmax=0.0, decay=DECAY)
+    dt = time.perf_counter() - t
+    return rows * K / dt, f"rows 0..{rows - 1} of the {M}x{K} matrix ({rows * K} elements), full row+col cast"
+
+
+def run_reference(args, rank: int, world: int) -> dict | None:
+    """The oracle as it stands, single-threaded, on bounded row slices of the same
+    matrix; the slice is sized so that warm-up + timed steps take about two minutes."""
+    if rank != 0:
+        return None
+    import oracle
+    from precision_quantization_row_b200 import inputs
+    oracle.build()
+    x = inputs.llm()
+    probe = oracle._bits(x[:16].contiguous())
+    t = time.perf_counter()
+    oracle.quantize(probe, absmax=0.0, decay=DECAY)
+    per_row = (time.perf_counter() - t) / 16
+    rows = int(120.0 / max(1, args.steps + args.warmup) / max(per_row, 1e-9)) // 16 * 16
+    rows = max(16, min(1024, rows))
+    samples = [oracle._bits(x[(i * rows) % M:(i * rows) % M + rows].contiguous()) for i in range(4)]
+    for i in range(args.warmup):
+        oracle.quantize(samples[i % 4], absmax=0.0, decay=DECAY)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        oracle.quantize(samples[i % 4], absmax=0.0, decay=DECAY)
+    secs = time.perf_counter() - t
+    value = rows * K * args.steps / secs
+    return {
+        "impl": "reference",
+        "metric": "NVFP4 per-token cast: elems/s, achieved HBM GB/s, % of B200 HBM peak",
+        "value": value, "unit": "elem/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16->nvfp4 (e2m1 codes, e4m3 scales, fp32 amax)", "data": "synthetic",
+        "config": {"workload": workload_name(M, K), "rows": M, "cols": K, "flags": "rowwise+columnwise",
+                   "absmax_decay": DECAY, "parallelism": "single CPU thread"},
+        "cpu_baseline": {"value": value, "unit": "elem/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows}-row slices ({rows * K} elements) of the {M}x{K} matrix per step"},
+        "e2e": {"value": value, "unit": "elem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rows", type=int, default=16384, help="rows of the activation (profiling runs)")
+    ap.add_argument("--cols", type=int, default=8192, help="columns of the activation (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        line = run_reference(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    dist = Dist(args.gpus)
+    try:
+        line = run_gpu(args, dist)
+        if line is not None and dist.world == 1 and not args.no_cpu_baseline:
+            rate, sample = oracle_sample_rate(8192)
+            line["cpu_baseline"] = {"value": rate, "unit": "elem/s", "cores": 1, "kind": "oracle",
+                                    "sample": sample}
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

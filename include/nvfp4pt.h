@@ -46,6 +46,12 @@
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
+#if defined(__GNUC__)
+#define NVFP4PT_API __attribute__((visibility("default")))
+#else
+#define NVFP4PT_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -72,13 +78,13 @@ enum { NVFP4PT_ROWWISE = 1, NVFP4PT_COLWISE = 2 };
 #define NVFP4PT_MAX_GROUPS 1024
 
 /* A constant, human-readable name of a status code. Never NULL. */
-const char* nvfp4pt_status_string(nvfp4pt_status status);
+NVFP4PT_API const char* nvfp4pt_status_string(nvfp4pt_status status);
 
 /* Bytes of device workspace a call with these sizes needs (num_groups = 1 for the
  * ungrouped and weight calls). The workspace holds per-call scratch (the observed
  * maxima of the absmax update and a device error word); it needs no initialisation
  * and its contents after a call are unspecified except for the error word. */
-size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
+NVFP4PT_API size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
 
 /*
  * nvfp4pt_quantize -- per-token cast of x[rows, cols] (PR #3045, Description and
@@ -94,7 +100,7 @@ size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
  *            with per-token scales the row amaxes are max-reduced to a scalar).
  * workspace  nvfp4pt_workspace_bytes(rows, cols, 1) bytes of device memory.
  */
-nvfp4pt_status nvfp4pt_quantize(const void* x_bf16, int64_t rows, int64_t cols, int flags,
+NVFP4PT_API nvfp4pt_status nvfp4pt_quantize(const void* x_bf16, int64_t rows, int64_t cols, int flags,
                                 uint8_t* q_row, uint8_t* sf_row, float* amax_row,
                                 uint8_t* q_col, uint8_t* sf_col, float* amax_col,
                                 float* absmax_buf, float decay,
@@ -118,7 +124,7 @@ nvfp4pt_status nvfp4pt_quantize(const void* x_bf16, int64_t rows, int64_t cols, 
  *            rows (0 for an empty group, which then only decays).
  * workspace  nvfp4pt_workspace_bytes(rows, cols, num_groups) bytes.
  */
-nvfp4pt_status nvfp4pt_quantize_grouped(const void* x_bf16, int64_t rows, int64_t cols,
+NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_grouped(const void* x_bf16, int64_t rows, int64_t cols,
                                         const int64_t* offsets_host, int num_groups, int flags,
                                         uint8_t* q_row, uint8_t* sf_row, float* amax_row,
                                         uint8_t* q_col, uint8_t* sf_col, float* amax_col,
@@ -136,7 +142,7 @@ nvfp4pt_status nvfp4pt_quantize_grouped(const void* x_bf16, int64_t rows, int64_
  * 1D cast. Weights are kept rowwise only (PR #3296, Description).
  * workspace  nvfp4pt_workspace_bytes(rows, cols, 1) bytes.
  */
-nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w_bf16, int64_t rows, int64_t cols,
+NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w_bf16, int64_t rows, int64_t cols,
                                           uint8_t* q_row, uint8_t* sf_row, float* amax_row,
                                           void* workspace, cudaStream_t stream);
 
@@ -146,7 +152,7 @@ nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w_bf16, int64_t rows, int6
  * (Observed = 0). Both pointers are device pointers; amax_vec holds n non-negative
  * fp32 values. No workspace; n <= 2^40.
  */
-nvfp4pt_status nvfp4pt_update_absmax(float* absmax_buf, const float* amax_vec, int64_t n,
+NVFP4PT_API nvfp4pt_status nvfp4pt_update_absmax(float* absmax_buf, const float* amax_vec, int64_t n,
                                      float decay, cudaStream_t stream);
 
 /*
@@ -156,7 +162,7 @@ nvfp4pt_status nvfp4pt_update_absmax(float* absmax_buf, const float* amax_vec, i
  * work; outputs of that call are then incomplete. Returns NVFP4PT_ERR_DEVICE if the
  * word is nonzero, NVFP4PT_OK otherwise (the word is stored in *word if non-NULL).
  */
-nvfp4pt_status nvfp4pt_workspace_error(const void* workspace, uint32_t* word, cudaStream_t stream);
+NVFP4PT_API nvfp4pt_status nvfp4pt_workspace_error(const void* workspace, uint32_t* word, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

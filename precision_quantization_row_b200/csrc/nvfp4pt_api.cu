@@ -1,0 +1,311 @@
+// Host side of the C ABI declared in include/nvfp4pt.h: argument checks, the TMA
+// descriptor of x, and the launches (zero -> amax pass -> encode pass, chained with
+// programmatic dependent launch on the caller's stream).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "nvfp4pt.h"
+#include "nvfp4pt_kernels.cuh"
+
+using namespace nvfp4pt;
+
+namespace {
+
+constexpr int64_t kMaxDim = int64_t(1) << 30;
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    int sm_count = 0;
+    int major = 0;
+    int minor = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+template <typename T>
+bool aligned16(const T* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device facts and one-time kernel attributes. Only called after all pure
+// argument checks have passed.
+nvfp4pt_status device_state(DeviceState** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4PT_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVFP4PT_ERR_CUDA;
+        if (d.major == 10 && d.minor == 0) {
+            const void* encoders[] = {(const void*)pass2_encode<1, false>, (const void*)pass2_encode<1, true>,
+                                      (const void*)pass2_encode<kMaxGroups, false>};
+            for (const void* f : encoders) {
+                if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPass2) != cudaSuccess ||
+                    cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+                    return NVFP4PT_ERR_CUDA;
+            }
+            if (!g_encode) {
+                cudaDriverEntryPointQueryResult q;
+                void* fn = nullptr;
+                if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || !fn)
+                    return NVFP4PT_ERR_CUDA;
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+        }
+        d.ready = true;
+    }
+    if (d.major != 10 || d.minor != 0) return NVFP4PT_ERR_ARCH;
+    *out = &d;
+    return NVFP4PT_OK;
+}
+
+nvfp4pt_status check_shape(int64_t rows, int64_t cols)
+{
+    if (rows <= 0 || cols <= 0 || rows > kMaxDim || cols > kMaxDim || rows % 16 || cols % 16)
+        return NVFP4PT_ERR_SHAPE;
+    return NVFP4PT_OK;
+}
+
+// x as a 2D bf16 tensor [rows, cols]; 128-row x 64-column boxes (128 bytes wide, the
+// span of the 128-byte swizzle); out-of-range elements read as zero.
+nvfp4pt_status encode_map(CUtensorMap* map, const void* x, int64_t rows, int64_t cols)
+{
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+}
+
+// Workspace layout: [0, 4) error word; [16, ...) observed maxima, one per buffer.
+uint32_t* ws_err(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
+float* ws_obs(void* ws) { return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 16); }
+int64_t pad4(int64_t n) { return (n + 3) & ~int64_t(3); }
+
+template <typename Kernel, typename Params>
+cudaError_t launch(Kernel kernel, int grid, int smem, cudaStream_t stream, const Params& p, bool pdl)
+{
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+cudaError_t launch_zero(cudaStream_t stream, const ZeroParams& z)
+{
+    int64_t total = 0;
+    for (int k = 0; k < 4; ++k) total += z.ptr[k] ? z.n4[k] : 0;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(148, (total + kThreads - 1) / kThreads));
+    return launch(pass0_zero, grid, 0, stream, z, false);
+}
+
+// The geometry and group tables of a call (offsets already validated).
+template <int MAXG>
+void fill_geometry(Geometry& geo, Groups<MAXG>& grp, int64_t rows, int64_t cols, const int64_t* off, int G,
+                   int sm_count)
+{
+    geo.rows = rows;
+    geo.cols = cols;
+    geo.ntc = (int32_t)((cols + kTile - 1) / kTile);
+    geo.num_groups = G;
+    int64_t bands = 0;
+    for (int g = 0; g < G; ++g) {
+        grp.band_start[g] = (int32_t)bands;
+        grp.row_off[g] = (int32_t)off[g];
+        bands += (off[g + 1] - off[g] + kTile - 1) / kTile;
+    }
+    grp.band_start[G] = (int32_t)bands;
+    grp.row_off[G] = (int32_t)off[G];
+    geo.total_tiles = bands * geo.ntc;
+    geo.num_ctas = (int32_t)std::min<int64_t>(geo.total_tiles, 2 * (int64_t)sm_count);
+    geo.pad_ = 0;
+}
+
+template <int MAXG>
+nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t* off, int G, int flags,
+                        uint8_t* q_row, uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col,
+                        float* amax_col, float* absmax, float decay, bool w2d, void* ws, cudaStream_t stream)
+{
+    DeviceState* dev = nullptr;
+    nvfp4pt_status st = device_state(&dev);
+    if (st != NVFP4PT_OK) return st;
+
+    const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
+    const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
+
+    P1Params<MAXG> p1;
+    std::memset(&p1, 0, sizeof p1);
+    fill_geometry<MAXG>(p1.geo, p1.grp, rows, cols, off, G, dev->sm_count);
+    p1.x = static_cast<const uint16_t*>(x);
+    p1.amax_row = do_row ? amax_row : nullptr;
+    p1.amax_col = do_col ? amax_col : nullptr;
+    p1.obs = absmax ? ws_obs(ws) : nullptr;
+
+    P2Params<MAXG> p2;
+    std::memset(&p2, 0, sizeof p2);
+    if ((st = encode_map(&p2.tmap, x, rows, cols)) != NVFP4PT_OK) return st;
+    p2.geo = p1.geo;
+    p2.grp = p1.grp;
+    p2.amax_row = amax_row;
+    p2.amax_col = amax_col;
+    p2.q_row = q_row;
+    p2.sf_row = sf_row;
+    p2.q_col = q_col;
+    p2.sf_col = sf_col;
+    p2.absmax = absmax;
+    p2.obs = ws_obs(ws);
+    p2.err = ws_err(ws);
+    p2.decay = decay;
+    p2.nbuf = absmax ? G : 0;
+    p2.flags = flags;
+
+    ZeroParams z;
+    std::memset(&z, 0, sizeof z);
+    if (do_row) { z.ptr[0] = reinterpret_cast<float4*>(amax_row); z.n4[0] = rows / 4; }
+    if (do_col) { z.ptr[1] = reinterpret_cast<float4*>(amax_col); z.n4[1] = (int64_t)G * cols / 4; }
+    if (absmax) { z.ptr[2] = reinterpret_cast<float4*>(ws_obs(ws)); z.n4[2] = pad4(G) / 4; }
+    z.err = ws_err(ws);
+
+    if (launch_zero(stream, z) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    cudaError_t e;
+    if (do_col) e = launch(pass1_amax<MAXG, true>, p1.geo.num_ctas, 0, stream, p1, true);
+    else e = launch(pass1_amax<MAXG, false>, p1.geo.num_ctas, 0, stream, p1, true);
+    if (e != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    if (w2d) e = launch(pass2_encode<MAXG, true>, p2.geo.num_ctas, kSmemPass2, stream, p2, true);
+    else e = launch(pass2_encode<MAXG, false>, p2.geo.num_ctas, kSmemPass2, stream, p2, true);
+    return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4pt_status_string(nvfp4pt_status s)
+{
+    switch (s) {
+    case NVFP4PT_OK: return "ok";
+    case NVFP4PT_ERR_NULL: return "a required pointer is NULL";
+    case NVFP4PT_ERR_SHAPE: return "rows and cols must be in (0, 2^30] and multiples of 16";
+    case NVFP4PT_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case NVFP4PT_ERR_GROUPS: return "invalid token groups (count or offsets)";
+    case NVFP4PT_ERR_ARCH: return "the current device is not sm_100 (B200)";
+    case NVFP4PT_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case NVFP4PT_ERR_FLAGS: return "flags must be a non-empty subset of ROWWISE|COLWISE";
+    case NVFP4PT_ERR_DEVICE: return "a kernel reported a device-side error";
+    }
+    return "unknown status";
+}
+
+size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups)
+{
+    (void)rows;
+    (void)cols;
+    const int64_t g = num_groups < 1 ? 1 : num_groups;
+    const int64_t bytes = 16 + 4 * pad4(g);
+    return (size_t)((bytes + 255) & ~int64_t(255));
+}
+
+nvfp4pt_status nvfp4pt_quantize(const void* x, int64_t rows, int64_t cols, int flags, uint8_t* q_row,
+                                uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                float* absmax_buf, float decay, void* workspace, cudaStream_t stream)
+{
+    const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
+    const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
+    if (!x || !workspace || (do_row && (!q_row || !sf_row || !amax_row)) ||
+        (do_col && (!q_col || !sf_col || !amax_col)))
+        return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = check_shape(rows, cols);
+    if (st != NVFP4PT_OK) return st;
+    if (flags & ~(NVFP4PT_ROWWISE | NVFP4PT_COLWISE) || !(do_row || do_col)) return NVFP4PT_ERR_FLAGS;
+    if (!aligned16(x) || !aligned16(static_cast<uint8_t*>(workspace)) || (absmax_buf && !aligned16(absmax_buf)) ||
+        (do_row && (!aligned16(q_row) || !aligned16(sf_row) || !aligned16(amax_row))) ||
+        (do_col && (!aligned16(q_col) || !aligned16(sf_col) || !aligned16(amax_col))))
+        return NVFP4PT_ERR_ALIGN;
+    const int64_t off[2] = {0, rows};
+    return run_cast<1>(x, rows, cols, off, 1, flags, q_row, sf_row, amax_row, q_col, sf_col, amax_col, absmax_buf,
+                       decay, false, workspace, stream);
+}
+
+nvfp4pt_status nvfp4pt_quantize_grouped(const void* x, int64_t rows, int64_t cols, const int64_t* offsets,
+                                        int num_groups, int flags, uint8_t* q_row, uint8_t* sf_row,
+                                        float* amax_row, uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                        float* absmax_bufs, float decay, void* workspace, cudaStream_t stream)
+{
+    const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
+    const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
+    if (!x || !workspace || !offsets || (do_row && (!q_row || !sf_row || !amax_row)) ||
+        (do_col && (!q_col || !sf_col || !amax_col)))
+        return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = check_shape(rows, cols);
+    if (st != NVFP4PT_OK) return st;
+    if (flags & ~(NVFP4PT_ROWWISE | NVFP4PT_COLWISE) || !(do_row || do_col)) return NVFP4PT_ERR_FLAGS;
+    if (!aligned16(x) || !aligned16(static_cast<uint8_t*>(workspace)) || (absmax_bufs && !aligned16(absmax_bufs)) ||
+        (do_row && (!aligned16(q_row) || !aligned16(sf_row) || !aligned16(amax_row))) ||
+        (do_col && (!aligned16(q_col) || !aligned16(sf_col) || !aligned16(amax_col))))
+        return NVFP4PT_ERR_ALIGN;
+    if (num_groups < 1 || num_groups > NVFP4PT_MAX_GROUPS || offsets[0] != 0 || offsets[num_groups] != rows)
+        return NVFP4PT_ERR_GROUPS;
+    for (int g = 0; g < num_groups; ++g)
+        if (offsets[g + 1] < offsets[g] || offsets[g] % 16) return NVFP4PT_ERR_GROUPS;
+    return run_cast<kMaxGroups>(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row, q_col, sf_col,
+                                amax_col, absmax_bufs, decay, false, workspace, stream);
+}
+
+nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w, int64_t rows, int64_t cols, uint8_t* q_row,
+                                          uint8_t* sf_row, float* amax_row, void* workspace, cudaStream_t stream)
+{
+    if (!w || !workspace || !q_row || !sf_row || !amax_row) return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = check_shape(rows, cols);
+    if (st != NVFP4PT_OK) return st;
+    if (!aligned16(w) || !aligned16(static_cast<uint8_t*>(workspace)) || !aligned16(q_row) || !aligned16(sf_row) ||
+        !aligned16(amax_row))
+        return NVFP4PT_ERR_ALIGN;
+    const int64_t off[2] = {0, rows};
+    return run_cast<1>(w, rows, cols, off, 1, NVFP4PT_ROWWISE, q_row, sf_row, amax_row, nullptr, nullptr, nullptr,
+                       nullptr, 0.0f, true, workspace, stream);
+}
+
+nvfp4pt_status nvfp4pt_update_absmax(float* buf, const float* v, int64_t n, float decay, cudaStream_t stream)
+{
+    if (!buf || (n > 0 && !v)) return NVFP4PT_ERR_NULL;
+    if (n < 0 || n > (int64_t(1) << 40)) return NVFP4PT_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(buf) & 3u) || (reinterpret_cast<uintptr_t>(v) & 3u)) return NVFP4PT_ERR_ALIGN;
+    DeviceState* dev = nullptr;
+    nvfp4pt_status st = device_state(&dev);
+    if (st != NVFP4PT_OK) return st;
+    update_absmax_kernel<<<1, 1024, 0, stream>>>(buf, v, n, decay);
+    return cudaGetLastError() == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+}
+
+nvfp4pt_status nvfp4pt_workspace_error(const void* workspace, uint32_t* word, cudaStream_t stream)
+{
+    if (!workspace) return NVFP4PT_ERR_NULL;
+    uint32_t w = 0;
+    if (cudaMemcpyAsync(&w, workspace, sizeof w, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return NVFP4PT_ERR_CUDA;
+    if (word) *word = w;
+    return w ? NVFP4PT_ERR_DEVICE : NVFP4PT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,351 @@
+// Device building blocks of the NVFP4 per-token cast for sm_100a.
+//
+// Everything here is one binary32 IEEE operation per step (the library is built
+// with -fmad=false, -prec-div=true, -ftz=false, and the arithmetic below uses the
+// explicitly rounded intrinsics), so that the codes are bit-identical to the
+// definition in include/nvfp4pt.h.
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+#include <cuda.h>
+
+namespace nvfp4pt {
+
+constexpr int kTile = 128;        // tile edge (rows and columns) of both passes
+constexpr int kThreads = 256;     // threads per CTA of both passes
+constexpr int kStages = 3;        // TMA stages of the encode pass
+constexpr int kBoxBytes = kTile * 64 * 2;     // one 128 x 64 bf16 TMA box (16 KB)
+constexpr int kStageBytes = 2 * kBoxBytes;    // a 128 x 128 bf16 tile (32 KB)
+constexpr int kMaxGroups = 1024;
+constexpr uint32_t kErrTmaTimeout = 1u;
+constexpr uint32_t kErrDrainTimeout = 2u;
+constexpr uint32_t kWaitLimit = 1u << 22;     // try_wait rounds before giving up (~seconds)
+
+// ------------------------------------------------------------------ geometry
+//
+// Both passes walk the same sequence of 128 x 128 tiles: for each token group g
+// (one group when ungrouped), its rows split into 128-row bands (the last band of a
+// group may be shorter, a multiple of 16), each band into ceil(cols/128) column
+// tiles. Tile t is band t / ntc, column tile t % ntc. CTA c of both passes owns the
+// same contiguous tile range; pass 2 walks it backwards so it starts on the tiles
+// pass 1 touched last (still in L2).
+
+struct Geometry {
+    int64_t rows;
+    int64_t cols;
+    int64_t total_tiles;
+    int32_t ntc;          // column tiles per band
+    int32_t num_groups;
+    int32_t num_ctas;     // CTAs of pass 1 and of pass 2 (same partition)
+    int32_t pad_;
+};
+
+template <int MAXG>
+struct Groups {
+    int32_t band_start[MAXG + 1];  // bands before group g (non-decreasing)
+    int32_t row_off[MAXG + 1];     // first row of group g; row_off[G] = rows
+};
+
+struct TileInfo {
+    int64_t band;   // global band index
+    int64_t r0;     // first row of the tile
+    int64_t c0;     // first column of the tile
+    int32_t g;      // token group
+    int32_t nr;     // valid rows (multiple of 16, 16..128)
+    int32_t nc;     // valid columns (multiple of 16, 16..128)
+    int32_t goff;   // first row of the group
+    int32_t grows;  // rows of the group
+};
+
+template <int MAXG>
+__device__ __forceinline__ TileInfo tile_info(const Geometry& geo, const Groups<MAXG>& grp, int64_t t)
+{
+    TileInfo ti;
+    ti.band = t / geo.ntc;
+    const int32_t ct = (int32_t)(t - ti.band * geo.ntc);
+    int g = 0;
+    if (MAXG > 1) {
+        int lo = 0, hi = geo.num_groups;  // band_start[lo] <= band < band_start[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if ((int64_t)grp.band_start[mid] <= ti.band) lo = mid; else hi = mid;
+        }
+        g = lo;
+    }
+    ti.g = g;
+    ti.goff = grp.row_off[g];
+    ti.grows = grp.row_off[g + 1] - grp.row_off[g];
+    const int64_t local_band = ti.band - grp.band_start[g];
+    ti.r0 = (int64_t)ti.goff + local_band * kTile;
+    const int64_t rem_r = (int64_t)grp.row_off[g + 1] - ti.r0;
+    ti.nr = (int32_t)(rem_r < kTile ? rem_r : kTile);
+    ti.c0 = (int64_t)ct * kTile;
+    const int64_t rem_c = geo.cols - ti.c0;
+    ti.nc = (int32_t)(rem_c < kTile ? rem_c : kTile);
+    return ti;
+}
+
+__device__ __forceinline__ void cta_tile_range(const Geometry& geo, int cta, int64_t& t0, int64_t& t1)
+{
+    t0 = (geo.total_tiles * cta) / geo.num_ctas;
+    t1 = (geo.total_tiles * (cta + 1)) / geo.num_ctas;
+}
+
+// ----------------------------------------------------- programmatic launch
+// The passes are chained with programmatic dependent launch: a dependent grid may
+// start while its predecessor drains, and must wait before touching its results.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// --------------------------------------------------------------- bf16 words
+// A 32-bit word holds two bf16 values: element 2j in the low half, 2j+1 in the high.
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Per-half max of magnitudes. The sign bits of the result are not meaningful (they
+// are the xor of the inputs' signs); callers clear them with & 0x7FFF7FFF.
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Larger of the two magnitudes held in w, as binary32 (exact: bf16 -> fp32).
+__device__ __forceinline__ float absmax_of_pair(uint32_t w)
+{
+    const uint32_t lo = w & 0x7FFFu;
+    const uint32_t hi = (w >> 16) & 0x7FFFu;
+    return __uint_as_float((lo > hi ? lo : hi) << 16);
+}
+
+// -------------------------------------------------------------- conversions
+
+// Byte of two E2M1 codes, round-to-nearest-even, saturating: `lo` -> bits 0-3,
+// `hi` -> bits 4-7. The hardware conversion puts its first source operand in the
+// high nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\t"
+        "cvt.u32.u8 %0, q;\n\t}"
+        : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// Eight products -> one 32-bit word of codes, element i in bits 4i..4i+3.
+__device__ __forceinline__ uint32_t e2m1x8(float y0, float y1, float y2, float y3,
+                                           float y4, float y5, float y6, float y7)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(r)
+        : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+    return r;
+}
+
+// Two E4M3 (e4m3fn) codes, round-to-nearest-even, saturating: `lo` -> bits 0-7,
+// `hi` -> bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// Exact value of the two E4M3 codes in the low 16 bits of `codes` (bits 0-7 -> lo).
+__device__ __forceinline__ void e4m3x2_decode(uint32_t codes, float& lo, float& hi)
+{
+    uint32_t h2;
+    const uint16_t c = (uint16_t)codes;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h2));
+}
+
+// ------------------------------------------------------------ block arithmetic
+
+// RN(b / 6) for every finite non-negative bf16 value b, in three operations:
+// q0 = RN(b * r), the exact remainder b - 6*q0 by one fused multiply-add, then one
+// correction step q0 + rem * r (the correction of Markstein's method, with the
+// reciprocal r = RN(1/6) fixed in advance). The result equals the IEEE quotient for
+// all 32640 such inputs; the library's probe entry checks that on the device.
+__device__ __forceinline__ float div6(float b)
+{
+    const float r = 0x1.555556p-3f;  // RN(1/6)
+    const float q0 = __fmul_rn(b, r);
+    const float rem = __fmaf_rn(-q0, 6.0f, b);
+    return __fmaf_rn(rem, r, q0);
+}
+
+// s_enc = 2688 / amax, 1 when amax == 0, clamped to FLT_MAX instead of overflowing.
+__device__ __forceinline__ float s_enc_of(float amax)
+{
+    if (amax == 0.0f) return 1.0f;
+    return fminf(__fdiv_rn(2688.0f, amax), FLT_MAX);
+}
+
+// enc = s_enc / float(sf), 0 when sf == 0, clamped to FLT_MAX.
+__device__ __forceinline__ float enc_of(uint32_t sf_code, float d, float s)
+{
+    return (sf_code & 0xFFu) ? fminf(__fdiv_rn(s, d), FLT_MAX) : 0.0f;
+}
+
+// Scale codes and multipliers of two blocks with block amaxes b0, b1 and outer
+// scales s0, s1. sf01 receives the two codes (block 0 in bits 0-7).
+__device__ __forceinline__ void block_pair_scales(float b0, float b1, float s0, float s1,
+                                                  uint32_t& sf01, float& e0, float& e1)
+{
+    const float u0 = __fmul_rn(div6(b0), s0);
+    const float u1 = __fmul_rn(div6(b1), s1);
+    sf01 = e4m3x2(u0, u1);
+    float d0, d1;
+    e4m3x2_decode(sf01, d0, d1);
+    e0 = enc_of(sf01, d0, s0);
+    e1 = enc_of(sf01 >> 8, d1, s1);
+}
+
+// Codes of the 8 elements held in 4 bf16 words with one multiplier.
+__device__ __forceinline__ uint32_t encode8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float e)
+{
+    return e2m1x8(__fmul_rn(bf16_lo(w0), e), __fmul_rn(bf16_hi(w0), e),
+                  __fmul_rn(bf16_lo(w1), e), __fmul_rn(bf16_hi(w1), e),
+                  __fmul_rn(bf16_lo(w2), e), __fmul_rn(bf16_hi(w2), e),
+                  __fmul_rn(bf16_lo(w3), e), __fmul_rn(bf16_hi(w3), e));
+}
+
+// ---------------------------------------------------------------- memory ops
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+// 16 bytes to global memory that is at least 8-byte aligned.
+__device__ __forceinline__ void stg16(uint8_t* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+        asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+    } else {
+        asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p), "r"(a), "r"(b) : "memory");
+        asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p + 8), "r"(c), "r"(d) : "memory");
+    }
+}
+
+__device__ __forceinline__ void stg8(uint8_t* p, uint32_t a, uint32_t b)
+{
+    asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p), "r"(a), "r"(b) : "memory");
+}
+
+// n (<= 4) bytes of v, low byte first, at any alignment.
+__device__ __forceinline__ void stg_bytes(uint8_t* p, uint32_t v, int n)
+{
+    if (n == 4 && (reinterpret_cast<uintptr_t>(p) & 3u) == 0) {
+        *reinterpret_cast<uint32_t*>(p) = v;
+    } else if (n == 2 && (reinterpret_cast<uintptr_t>(p) & 1u) == 0) {
+        *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
+    } else {
+        for (int i = 0; i < n; ++i) p[i] = (uint8_t)(v >> (8 * i));
+    }
+}
+
+// Non-negative binary32 maxima are combined as their bit patterns (order-preserving
+// for non-negative values); the targets start at +0.
+__device__ __forceinline__ void red_max_f32(float* p, uint32_t bits)
+{
+    atomicMax(reinterpret_cast<unsigned int*>(p), bits);
+}
+
+// ------------------------------------------------------------ mbarrier + TMA
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of the barrier to complete, giving up after kWaitLimit
+// rounds (each try_wait round may itself suspend the thread for a while).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+{
+    for (uint32_t i = 0; i < kWaitLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// One 2D tiled TMA load (box = the tensor map's box) into shared memory, completing
+// on `bar`. x is the column (innermost) coordinate, a multiple of 64 elements.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map)
+{
+    asm volatile("prefetch.tensormap [%0];" :: "l"(map) : "memory");
+}
+
+// Byte offset, inside a 128-row x 128-byte box loaded with 128-byte swizzling, of the
+// 16-byte chunk `chunk` of row `row`: the chunk index is xor-ed with row % 8.
+__device__ __forceinline__ uint32_t swz128(int row, int chunk)
+{
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+}  // namespace nvfp4pt

@@ -1,0 +1,130 @@
+// Diagnostic kernels (include/nvfp4pt_probe.h): the cast's device conversions run
+// over whole input domains so the tests can compare them with the CPU definition.
+#include "nvfp4pt_probe.h"
+#include "nvfp4pt_device.cuh"
+
+using namespace nvfp4pt;
+
+namespace {
+
+constexpr uint32_t kChunk = 4096;
+
+__device__ __forceinline__ uint32_t probe_code(int which, uint32_t bits)
+{
+    const float f = __uint_as_float(bits);
+    return which == 0 ? (e2m1x2(f, 0.0f) & 0xFu) : (e4m3x2(f, 0.0f) & 0xFFu);
+}
+
+// Ranges: [0, 0x7F800000] and [0x80000000, 0xFF800000], each 0x7F800001 patterns.
+__global__ void transitions_kernel(int which, uint32_t* out, uint32_t cap, uint32_t* count)
+{
+    const uint64_t per_range = 0x7F800001ull;
+    const uint64_t chunks_per_range = (per_range + kChunk - 1) / kChunk;
+    const uint64_t total_chunks = 2 * chunks_per_range;
+    for (uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total_chunks;
+         c += (uint64_t)gridDim.x * blockDim.x) {
+        const uint64_t range = c / chunks_per_range;
+        const uint64_t first = (c % chunks_per_range) * kChunk;
+        const uint64_t last = first + kChunk < per_range ? first + kChunk : per_range;
+        const uint32_t base = range ? 0x80000000u : 0u;
+        uint32_t prev = first == 0 ? 0xFFFFFFFFu : probe_code(which, base + (uint32_t)(first - 1));
+        for (uint64_t i = first; i < last; ++i) {
+            const uint32_t bits = base + (uint32_t)i;
+            const uint32_t code = probe_code(which, bits);
+            if (code != prev) {
+                const uint32_t slot = atomicAdd(count, 1u);
+                if (slot < cap) {
+                    out[2 * (uint64_t)slot] = bits;
+                    out[2 * (uint64_t)slot + 1] = code;
+                }
+            }
+            prev = code;
+        }
+    }
+}
+
+__global__ void pairs_kernel(const float* in, int64_t n, uint32_t* out)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float lo = in[2 * i], hi = in[2 * i + 1];
+        out[i] = (e2m1x2(lo, hi) & 0xFFu) | (e4m3x2(lo, hi) << 16);
+    }
+}
+
+__global__ void decode_kernel(float* out)
+{
+    const uint32_t c = threadIdx.x;
+    float lo, hi;
+    e4m3x2_decode(c, lo, hi);
+    out[c] = lo;
+    e4m3x2_decode(c << 8, lo, hi);
+    out[256 + c] = hi;
+}
+
+__global__ void div6_kernel(float* out)
+{
+    const uint32_t h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h < 0x7F80u) out[h] = div6(__uint_as_float(h << 16));
+}
+
+nvfp4pt_status arch_ok()
+{
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return NVFP4PT_ERR_CUDA;
+    return (major == 10 && minor == 0) ? NVFP4PT_OK : NVFP4PT_ERR_ARCH;
+}
+
+nvfp4pt_status last()
+{
+    return cudaGetLastError() == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4pt_status nvfp4pt_probe_transitions(int which, uint32_t* out, uint32_t capacity, uint32_t* count,
+                                         cudaStream_t stream)
+{
+    if (!out || !count) return NVFP4PT_ERR_NULL;
+    if (which != 0 && which != 1) return NVFP4PT_ERR_FLAGS;
+    nvfp4pt_status st = arch_ok();
+    if (st != NVFP4PT_OK) return st;
+    if (cudaMemsetAsync(count, 0, sizeof(uint32_t), stream) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    transitions_kernel<<<148 * 8, 256, 0, stream>>>(which, out, capacity, count);
+    return last();
+}
+
+nvfp4pt_status nvfp4pt_probe_pairs(const float* in, int64_t n, uint32_t* out, cudaStream_t stream)
+{
+    if (!in || !out) return NVFP4PT_ERR_NULL;
+    if (n <= 0) return NVFP4PT_ERR_SHAPE;
+    nvfp4pt_status st = arch_ok();
+    if (st != NVFP4PT_OK) return st;
+    const int64_t blocks = (n + 255) / 256;
+    pairs_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(in, n, out);
+    return last();
+}
+
+nvfp4pt_status nvfp4pt_probe_e4m3_decode(float* out, cudaStream_t stream)
+{
+    if (!out) return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = arch_ok();
+    if (st != NVFP4PT_OK) return st;
+    decode_kernel<<<1, 256, 0, stream>>>(out);
+    return last();
+}
+
+nvfp4pt_status nvfp4pt_probe_div6(float* out, cudaStream_t stream)
+{
+    if (!out) return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = arch_ok();
+    if (st != NVFP4PT_OK) return st;
+    div6_kernel<<<(0x7F80 + 255) / 256, 256, 0, stream>>>(out);
+    return last();
+}
+
+}  // extern "C"

@@ -1,0 +1,139 @@
+"""Helpers of the GPU parity tests: run the CUDA path, run the oracle (in parallel
+over exact sub-problems for the large workloads), compare element by element.
+
+Sub-problems used for the parallel oracle are exact restrictions of the cast: the
+rowwise outputs of a row range depend only on those rows; the columnwise outputs of
+a column range only on those columns; each token group's columnwise outputs only on
+the group's rows; the 2D weight outputs of a run of 16-row bands only on those rows.
+"""
+from __future__ import annotations
+
+import concurrent.futures as cf
+import multiprocessing as mp
+import os
+import tempfile
+
+import numpy as np
+import torch
+
+import oracle
+
+ROWWISE, COLWISE = 1, 2
+
+
+def to_np(out: dict) -> dict:
+    return {k: v.detach().cpu().numpy() for k, v in out.items()}
+
+
+def bits_of(x: torch.Tensor) -> np.ndarray:
+    return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def compare(got: dict, want: dict, keys=None, label="") -> None:
+    """Bit-exact comparison; floats compared as their bit patterns."""
+    keys = keys or sorted(want)
+    for k in keys:
+        g = np.atleast_1d(np.asarray(got[k]))
+        w = np.atleast_1d(np.asarray(want[k], dtype=np.float32 if np.isscalar(want[k]) else None))
+        assert g.shape == w.shape or g.size == w.size, (label, k, g.shape, w.shape)
+        g = g.reshape(w.shape)
+        if w.dtype == np.float32:
+            g, w = g.view(np.uint32), w.view(np.uint32)
+        bad = np.nonzero(g != w)
+        n = bad[0].size
+        if n:
+            idx = tuple(b[:8] for b in bad)
+            raise AssertionError(f"{label} {k}: {n} of {w.size} differ; first at {list(zip(*idx))}: "
+                                 f"got {g[idx]} want {w[idx]}")
+
+
+# ------------------------------------------------------------ parallel oracle
+
+def _worker(task):
+    kind, path, a, b, extra = task
+    x = np.load(path, mmap_mode="r")
+    if kind == "rows":
+        return kind, a, b, oracle.quantize(np.ascontiguousarray(x[a:b]), flags=ROWWISE)
+    if kind == "cols":
+        return kind, a, b, oracle.quantize(np.ascontiguousarray(x[:, a:b]), flags=COLWISE)
+    if kind == "group":
+        return kind, a, b, oracle.quantize(np.ascontiguousarray(x[a:b]), flags=COLWISE)
+    if kind == "w2d":
+        return kind, a, b, oracle.quantize_weight_2d(np.ascontiguousarray(x[a:b]))
+    raise ValueError(kind)
+
+
+def _pool(n_tasks):
+    workers = max(1, min(n_tasks, os.cpu_count() or 1, 32))
+    return cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn"))
+
+
+def _split(n, parts, align=16):
+    step = max(align, -(-n // parts) // align * align)
+    return [(a, min(n, a + step)) for a in range(0, n, step)]
+
+
+def oracle_quantize_parallel(x: torch.Tensor, flags=ROWWISE | COLWISE, offsets=None, parts=None) -> dict:
+    """The oracle's cast of x, computed over exact sub-problems in a spawn pool."""
+    xb = bits_of(x)
+    M, K = xb.shape
+    parts = parts or max(1, min(32, os.cpu_count() or 1)) * 2
+    out = {"amax_row": np.zeros(M, np.float32)}
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "x.npy")
+        np.save(path, xb)
+        tasks = [("rows", path, a, b, None) for a, b in _split(M, parts)]
+        if flags & ROWWISE:
+            out["q_row"] = np.zeros((M, K // 2), np.uint8)
+            out["sf_row"] = np.zeros((M, K // 16), np.uint8)
+        if flags & COLWISE:
+            if offsets is None:
+                out["q_col"] = np.zeros((K, M // 2), np.uint8)
+                out["sf_col"] = np.zeros((K, M // 16), np.uint8)
+                out["amax_col"] = np.zeros(K, np.float32)
+                tasks += [("cols", path, a, b, None) for a, b in _split(K, parts)]
+            else:
+                G = len(offsets) - 1
+                out["q_col"] = np.zeros(K * M // 2, np.uint8)
+                out["sf_col"] = np.zeros(K * M // 16, np.uint8)
+                out["amax_col"] = np.zeros((G, K), np.float32)
+                tasks += [("group", path, int(offsets[g]), int(offsets[g + 1]), g)
+                          for g in range(G) if offsets[g + 1] > offsets[g]]
+        with _pool(len(tasks)) as ex:
+            futs = {ex.submit(_worker, t): t for t in tasks}
+            for f in cf.as_completed(futs):
+                kind, a, b, r = f.result()
+                g = futs[f][4]
+                if kind == "rows":
+                    out["amax_row"][a:b] = r["amax_row"]
+                    if flags & ROWWISE:
+                        out["q_row"][a:b] = r["q_row"]
+                        out["sf_row"][a:b] = r["sf_row"]
+                elif kind == "cols":
+                    out["q_col"][a:b] = r["q_col"]
+                    out["sf_col"][a:b] = r["sf_col"]
+                    out["amax_col"][a:b] = r["amax_col"]
+                else:  # group
+                    out["q_col"][K * a // 2:K * b // 2] = r["q_col"].ravel()
+                    out["sf_col"][K * a // 16:K * b // 16] = r["sf_col"].ravel()
+                    out["amax_col"][g] = r["amax_col"]
+    if not flags & ROWWISE:
+        out.pop("amax_row")
+    return out
+
+
+def oracle_weight_2d_parallel(w: torch.Tensor, parts=None) -> dict:
+    wb = bits_of(w)
+    N, K = wb.shape
+    parts = parts or max(1, min(32, os.cpu_count() or 1)) * 2
+    out = {"q_row": np.zeros((N, K // 2), np.uint8), "sf_row": np.zeros((N, K // 16), np.uint8),
+           "amax_row": np.zeros(N, np.float32)}
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "w.npy")
+        np.save(path, wb)
+        tasks = [("w2d", path, a, b, None) for a, b in _split(N, parts)]
+        with _pool(len(tasks)) as ex:
+            for kind, a, b, r in ex.map(_worker, tasks):
+                for k in out:
+                    out[k][a:b] = r[k]
+    return out

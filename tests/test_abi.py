@@ -1,0 +1,133 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the headers
+declare, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import precision_quantization_row_b200 as nv
+from precision_quantization_row_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return nv.lib()
+
+
+def _declared():
+    names = []
+    for h in ("nvfp4pt.h", "nvfp4pt_probe.h"):
+        with open(os.path.join(ROOT, "include", h)) as f:
+            names += re.findall(r"NVFP4PT_API\s+[\w\s\*]+?\b(nvfp4pt_\w+)\s*\(", f.read())
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(nv.EXPORTS)
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert L.nvfp4pt_status_string(code)
+    assert L.nvfp4pt_status_string(99) == b"unknown status"
+
+
+def test_workspace_bytes(L):
+    assert nv.workspace_bytes(16, 16, 1) >= 20
+    assert nv.workspace_bytes(65536, 7168, 64) >= 16 + 4 * 64
+    assert nv.workspace_bytes(16, 16, 1024) >= 16 + 4 * 1024
+    assert nv.workspace_bytes(16, 16, 7) % 256 == 0
+
+
+class _Host:
+    """A 16-byte aligned host scratch area standing in for pointers (never dereferenced:
+    every call below fails validation before any device access)."""
+
+    def __init__(self):
+        self.buf = ctypes.create_string_buffer(1 << 12)
+        self.a = (ctypes.addressof(self.buf) + 15) // 16 * 16
+
+    def p(self, off=0):
+        return ctypes.c_void_p(self.a + off)
+
+
+F0 = ctypes.c_float(0.0)
+
+
+def test_quantize_rejections(L):
+    h = _Host()
+    P = h.p
+    q = lambda x, r, c, fl, *o: L.nvfp4pt_quantize(x, r, c, fl, *o, None, F0, P(), None)
+    ok7 = [P()] * 6
+    assert q(None, 16, 16, 3, *ok7) == 1
+    assert q(P(), 16, 16, 1, None, P(), P(), None, None, None) == 1            # rowwise output missing
+    assert q(P(), 16, 16, 2, P(), P(), P(), P(), None, P()) == 1                # colwise output missing
+    assert L.nvfp4pt_quantize(P(), 16, 16, 3, *ok7, None, F0, None, None) == 1  # workspace
+    for r, c in [(15, 16), (16, 8), (0, 16), (16, -16), (1 << 31, 16)]:
+        assert q(P(), r, c, 3, *ok7) == 2, (r, c)
+    for fl in (0, 4, 7):
+        assert q(P(), 16, 16, fl, *ok7) == 7, fl
+    assert q(P(8), 16, 16, 3, *ok7) == 3
+    assert q(P(), 16, 16, 3, P(4), P(), P(), P(), P(), P()) == 3
+    assert q(P(), 16, 16, 3, P(), P(), P(), P(), P(), P(2)) == 3
+    assert L.nvfp4pt_quantize(P(), 16, 16, 3, *ok7, P(4), F0, P(), None) == 3  # absmax buffer alignment
+    # rowwise only: columnwise pointers are ignored, even if misaligned
+    assert q(P(), 16, 16, 1, P(), P(), P(), P(3), None, None) not in (1, 3)
+
+
+def test_grouped_rejections(L):
+    h = _Host()
+    P = h.p
+
+    def g(offs, G=None, rows=64):
+        arr = (ctypes.c_int64 * len(offs))(*offs)
+        G = len(offs) - 1 if G is None else G
+        return L.nvfp4pt_quantize_grouped(P(), rows, 32, arr, G, 3, *[P()] * 6, None, F0, P(), None)
+
+    assert L.nvfp4pt_quantize_grouped(P(), 64, 32, None, 1, 3, *[P()] * 6, None, F0, P(), None) == 1
+    assert g([0, 64], G=0) == 4
+    assert g([0, 64], G=1025) == 4
+    assert g([16, 64]) == 4          # does not start at 0
+    assert g([0, 48]) == 4           # does not end at rows
+    assert g([0, 32, 16, 64]) == 4   # decreasing
+    assert g([0, 8, 64]) == 4        # not a multiple of 16
+    # valid offsets (including empty groups) pass validation and fail only at the CUDA step here
+    assert g([0, 0, 32, 32, 64]) in (5, 6)
+
+
+def test_weight_and_absmax_rejections(L):
+    h = _Host()
+    P = h.p
+    assert L.nvfp4pt_quantize_weight_2d(None, 16, 16, P(), P(), P(), P(), None) == 1
+    assert L.nvfp4pt_quantize_weight_2d(P(), 16, 17, P(), P(), P(), P(), None) == 2
+    assert L.nvfp4pt_quantize_weight_2d(P(), 16, 16, P(1), P(), P(), P(), None) == 3
+    assert L.nvfp4pt_update_absmax(None, P(), 4, F0, None) == 1
+    assert L.nvfp4pt_update_absmax(P(), None, 4, F0, None) == 1
+    assert L.nvfp4pt_update_absmax(P(), P(), -1, F0, None) == 2
+    assert L.nvfp4pt_update_absmax(P(2), P(), 4, F0, None) == 3
+    assert L.nvfp4pt_workspace_error(None, None, None) == 1
+
+
+def test_probe_rejections(L):
+    h = _Host()
+    P = h.p
+    assert L.nvfp4pt_probe_transitions(0, None, 8, P(), None) == 1
+    assert L.nvfp4pt_probe_transitions(2, P(), 8, P(), None) == 7
+    assert L.nvfp4pt_probe_pairs(P(), 0, P(), None) == 2
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros((16, 16), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        nv.quantize(x)
+    with pytest.raises(TypeError):
+        nv.quantize_weight_2d(x)

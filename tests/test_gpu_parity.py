@@ -1,0 +1,216 @@
+"""The CUDA path (through the C ABI) against the oracle, element by element, bit-exact.
+
+Codes and scales are integers and amax values / running buffers are exact (a max
+of bf16 values; one binary32 multiply), so the bar is bit-equality everywhere.
+The workloads are the five synthetic configurations (tiny, dense, LLM-sized,
+MoE grouped, 2D weight + calibration stream) at full size, plus ragged shapes
+that span several tiles with partial tails, and the degenerate inputs of the
+method (zero rows, signed zeros, bf16-subnormal rows, huge dynamic range).
+"""
+import numpy as np
+import pytest
+import torch
+
+import precision_quantization_row_b200 as nv
+from precision_quantization_row_b200 import inputs
+from parity_util import compare, oracle_quantize_parallel, oracle_weight_2d_parallel, to_np
+
+pytestmark = pytest.mark.gpu
+RC = nv.ROWWISE | nv.COLWISE
+
+
+def gpu_cast(x, flags=RC, absmax=None, decay=0.0):
+    xd = x.cuda()
+    buf = None if absmax is None else torch.tensor([absmax], dtype=torch.float32, device="cuda")
+    ws = nv.new_workspace(*x.shape, device="cuda")
+    out = to_np(nv.quantize(xd, flags=flags, absmax=buf, decay=decay, workspace=ws))
+    assert nv.workspace_error(ws) == 0
+    if buf is not None:
+        out["absmax"] = buf.cpu().numpy()
+    return out
+
+
+# ----------------------------------------------------------------- configs
+
+def test_tiny_config_and_absmax_stream(orc):
+    """Tiny: [256, 512], outlier rows 7 and 100, zero row 3; buffer over seeds 0..9 at decay 0.9."""
+    gbuf = torch.zeros(1, dtype=torch.float32, device="cuda")
+    obuf = 0.0
+    ws = nv.new_workspace(256, 512, device="cuda")
+    for seed in range(10):
+        x = inputs.tiny(seed)
+        got = to_np(nv.quantize(x.cuda(), absmax=gbuf, decay=0.9, workspace=ws))
+        want = orc.quantize(x, absmax=obuf, decay=0.9)
+        obuf = want.pop("absmax")
+        compare(got, want, label=f"tiny seed {seed}")
+        assert np.float32(gbuf.item()).view(np.uint32) == np.float32(obuf).view(np.uint32)
+    assert nv.workspace_error(ws) == 0
+
+
+def test_dense_config(orc):
+    x = inputs.dense()
+    compare(gpu_cast(x), oracle_quantize_parallel(x), label="dense")
+
+
+@pytest.mark.slow
+def test_llm_config_full(orc):
+    """The headline workload, in the call the benchmark times."""
+    x = inputs.llm()
+    got = gpu_cast(x, absmax=0.0, decay=0.99)
+    want = oracle_quantize_parallel(x)
+    compare(got, want, label="llm")
+    assert got["absmax"][0] == want["amax_row"].max()
+
+
+@pytest.mark.slow
+def test_moe_grouped_config_full(orc):
+    x, offsets = inputs.moe()
+    G = len(offsets) - 1
+    bufs = torch.full((G,), 1.0, dtype=torch.float32, device="cuda")
+    ws = nv.new_workspace(*x.shape, G, device="cuda")
+    got = to_np(nv.quantize_grouped(x.cuda(), offsets, absmax=bufs, decay=0.5, workspace=ws))
+    assert nv.workspace_error(ws) == 0
+    want = oracle_quantize_parallel(x, offsets=offsets)
+    compare(got, want, label="moe")
+    obs = np.array([want["amax_col"][g].max() for g in range(G)], np.float32)
+    assert np.array_equal(bufs.cpu().numpy(), np.maximum(np.float32(0.5), obs))
+
+
+@pytest.mark.slow
+def test_weight_2d_config_full(orc):
+    w = inputs.weight()
+    ws = nv.new_workspace(*w.shape, device="cuda")
+    got = to_np(nv.quantize_weight_2d(w.cuda(), workspace=ws))
+    assert nv.workspace_error(ws) == 0
+    compare(got, oracle_weight_2d_parallel(w), label="weight2d")
+
+
+@pytest.mark.slow
+def test_calibration_stream(orc):
+    """200 activations with sigma_t = 1 + 0.5 sin(t/20) through the fused cast and the
+    decayed buffer (decay 0.99): buffer and amax vectors at every step, codes and
+    scales at t = 0, 99, 199."""
+    M, K = 8192, 4096
+    gbuf = torch.zeros(1, dtype=torch.float32, device="cuda")
+    ws = nv.new_workspace(M, K, device="cuda")
+    out = None
+    obuf = np.float32(0.0)
+    for t in range(200):
+        a = inputs.calib_step(t, M, K)
+        out = nv.quantize(a, absmax=gbuf, decay=0.99, out=out, workspace=ws)
+        a_h = a.cpu()
+        want_r = orc.amax_rows(a_h)
+        want_c = orc.amax_cols(a_h)
+        obuf = np.float32(orc.update_absmax(float(obuf), want_r, 0.99))
+        got = to_np({k: out[k] for k in ("amax_row", "amax_col")})
+        compare(got, {"amax_row": want_r, "amax_col": want_c}, label=f"calib t={t}")
+        assert np.float32(gbuf.item()).view(np.uint32) == obuf.view(np.uint32), t
+        if t in (0, 99, 199):
+            compare(to_np(out), oracle_quantize_parallel(a_h), label=f"calib cast t={t}")
+    assert nv.workspace_error(ws) == 0
+
+
+# --------------------------------------------------------- shapes and edges
+
+SHAPES = [(16, 16), (16, 32), (32, 16), (48, 80), (144, 272), (256, 48), (128, 128), (272, 144),
+          (1040, 1056), (16, 4096), (4096, 16), (400, 656)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}x{s[1]}")
+@pytest.mark.parametrize("kind", ["normal", "wide"])
+def test_shapes(orc, shape, kind):
+    x = inputs.random_shape(hash(shape) % 1000, *shape, kind)
+    compare(gpu_cast(x, absmax=3.0, decay=0.5), orc.quantize(x, absmax=3.0, decay=0.5), label=f"{shape} {kind}")
+
+
+@pytest.mark.parametrize("kind", ["zeros", "signed_zero", "tiny", "wide"])
+def test_degenerate_inputs(orc, kind):
+    x = inputs.random_shape(11, 272, 400, kind)
+    compare(gpu_cast(x, absmax=0.0, decay=1.0), orc.quantize(x, absmax=0.0, decay=1.0), label=kind)
+
+
+def test_mixed_rows(orc):
+    """Zero rows, subnormal rows, single-nonzero rows and huge rows in one matrix."""
+    x = inputs.random_shape(12, 256, 384, "normal").float()
+    x[0] = 0.0
+    x[1] = x[1] * 1e-39
+    x[2] = 0.0
+    x[2, 77] = -3.0e-5
+    x[3] = x[3] / x[3].abs().max() * 3.0e38  # largest finite magnitudes (inf is out of contract)
+    x[:, 5] = 0.0
+    x[:, 6] = -0.0
+    x = x.to(torch.bfloat16)
+    compare(gpu_cast(x), orc.quantize(x), label="mixed")
+
+
+@pytest.mark.parametrize("flags", [nv.ROWWISE, nv.COLWISE])
+def test_single_direction(orc, flags):
+    x = inputs.random_shape(13, 400, 272, "wide")
+    got = gpu_cast(x, flags=flags, absmax=2.0, decay=0.25)
+    want = orc.quantize(x, flags=flags, absmax=2.0, decay=0.25)
+    if not flags & nv.ROWWISE:
+        want.pop("amax_row")
+    compare(got, want, label=f"flags {flags}")
+
+
+def test_repeated_calls_reuse_buffers(orc):
+    """Outputs and workspace reused across calls of different inputs: nothing stale."""
+    ws = nv.new_workspace(1040, 1056, device="cuda")
+    out = None
+    for seed, kind in [(1, "wide"), (2, "zeros"), (3, "normal")]:
+        x = inputs.random_shape(seed, 1040, 1056, kind)
+        out = nv.quantize(x.cuda(), out=out, workspace=ws)
+        compare(to_np(out), orc.quantize(x), label=f"reuse {seed}")
+
+
+def test_update_absmax(orc):
+    rng = np.random.default_rng(14)
+    for n in (0, 1, 1000, 1 << 20):
+        v = np.abs(rng.standard_normal(n)).astype(np.float32) * 7
+        buf = torch.tensor([5.0], dtype=torch.float32, device="cuda")
+        nv.update_absmax(buf, torch.from_numpy(v).cuda(), 0.75)
+        assert np.float32(buf.item()) == np.float32(orc.update_absmax(5.0, v, 0.75)), n
+
+
+# ------------------------------------------------------------------ grouped
+
+GROUPINGS = [
+    (64, [0, 64]),
+    (256, [0, 0, 128, 128, 256]),
+    (400, [0, 16, 48, 48, 400]),
+    (272, [0, 144, 160, 272]),
+    (1024, [0, 128, 256, 384, 512, 640, 768, 896, 1024]),
+]
+
+
+@pytest.mark.parametrize("rows,offsets", GROUPINGS)
+def test_grouped(orc, rows, offsets):
+    x = inputs.random_shape(rows, rows, 272, "wide")
+    G = len(offsets) - 1
+    bufs = torch.full((G,), 2.0, dtype=torch.float32, device="cuda")
+    ws = nv.new_workspace(rows, 272, G, device="cuda")
+    got = to_np(nv.quantize_grouped(x.cuda(), offsets, absmax=bufs, decay=0.5, workspace=ws))
+    assert nv.workspace_error(ws) == 0
+    want = orc.quantize_grouped(x, offsets, absmax=np.full(G, 2.0, np.float32), decay=0.5)
+    got["absmax"] = bufs.cpu().numpy()
+    compare(got, want, label=f"grouped {offsets}")
+
+
+def test_grouped_many_groups(orc):
+    rng = np.random.default_rng(15)
+    G = 1024
+    sizes = rng.multinomial(200, [1 / G] * G) * 16
+    offsets = np.concatenate([[0], np.cumsum(sizes)])
+    rows = int(offsets[-1])
+    x = inputs.random_shape(16, rows, 64, "wide")
+    got = to_np(nv.quantize_grouped(x.cuda(), offsets))
+    compare(got, orc.quantize_grouped(x, offsets), label="1024 groups")
+
+
+# --------------------------------------------------------------- weight 2D
+
+@pytest.mark.parametrize("shape", [(16, 16), (48, 80), (272, 400), (1040, 1056)])
+def test_weight_2d(orc, shape):
+    w = inputs.random_shape(17, *shape, "wide")
+    got = to_np(nv.quantize_weight_2d(w.cuda()))
+    compare(got, orc.quantize_weight_2d(w), label=f"w2d {shape}")
