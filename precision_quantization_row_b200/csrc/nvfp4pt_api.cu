@@ -9,6 +9,7 @@
 
 #include "nvfp4pt.h"
 #include "nvfp4pt_kernels.cuh"
+#include "nvfp4pt_rowpass.cuh"
 
 using namespace nvfp4pt;
 
@@ -95,12 +96,13 @@ float* ws_obs(void* ws) { return reinterpret_cast<float*>(static_cast<uint8_t*>(
 int64_t pad4(int64_t n) { return (n + 3) & ~int64_t(3); }
 
 template <typename Kernel, typename Params>
-cudaError_t launch(Kernel kernel, int grid, int smem, cudaStream_t stream, const Params& p, bool pdl)
+cudaError_t launch(Kernel kernel, int grid, int smem, cudaStream_t stream, const Params& p, bool pdl,
+                   int threads = kThreads)
 {
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -122,7 +124,7 @@ cudaError_t launch_zero(cudaStream_t stream, const ZeroParams& z)
 // The geometry and group tables of a call (offsets already validated).
 template <int MAXG>
 void fill_geometry(Geometry& geo, Groups<MAXG>& grp, int64_t rows, int64_t cols, const int64_t* off, int G,
-                   int sm_count)
+                   int num_ctas_max, int interleave)
 {
     geo.rows = rows;
     geo.cols = cols;
@@ -137,8 +139,38 @@ void fill_geometry(Geometry& geo, Groups<MAXG>& grp, int64_t rows, int64_t cols,
     grp.band_start[G] = (int32_t)bands;
     grp.row_off[G] = (int32_t)off[G];
     geo.total_tiles = bands * geo.ntc;
-    geo.num_ctas = (int32_t)std::min<int64_t>(geo.total_tiles, 2 * (int64_t)sm_count);
-    geo.pad_ = 0;
+    const int64_t ranges = std::max<int64_t>(1, std::min<int64_t>(geo.total_tiles, num_ctas_max / interleave));
+    geo.interleave = interleave;
+    geo.num_ctas = (int32_t)(ranges * interleave);
+}
+
+// Shape of the row pass for `cols` columns (cols <= kRowPassMaxCols): blocks per thread
+// and row (bt), threads per row (tpr), rows per sweep (rps) and sweeps per batch (S).
+constexpr int64_t kRowPassMaxCols = 16384;
+struct RowShape {
+    int bpr, bt, tpr, rps, S;
+};
+RowShape row_shape(int64_t cols)
+{
+    RowShape r;
+    r.bpr = (int)(cols / 16);
+    r.bt = (r.bpr + kRowThreads - 1) / kRowThreads;
+    const int per = (r.bpr + r.bt - 1) / r.bt;
+    r.tpr = (per + 31) / 32 * 32;
+    r.rps = 1;
+    while (r.rps * 2 <= 16 && r.rps * 2 * r.tpr <= kRowThreads) r.rps *= 2;
+    r.S = r.bt == 2 ? 2 : std::min(4, 16 / r.rps);
+    return r;
+}
+
+template <int MAXG>
+cudaError_t launch_rowpass(const RowShape& rs, const RowParams<MAXG>& rp, cudaStream_t stream)
+{
+    const int grid = rp.num_ctas;
+    if (rs.bt == 2) return launch(rowpass<MAXG, 2, 2>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.S == 4) return launch(rowpass<MAXG, 1, 4>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.S == 2) return launch(rowpass<MAXG, 1, 2>, grid, 0, stream, rp, true, kRowThreads);
+    return launch(rowpass<MAXG, 1, 1>, grid, 0, stream, rp, true, kRowThreads);
 }
 
 template <int MAXG>
@@ -152,20 +184,13 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
 
     const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
     const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
-
-    P1Params<MAXG> p1;
-    std::memset(&p1, 0, sizeof p1);
-    fill_geometry<MAXG>(p1.geo, p1.grp, rows, cols, off, G, dev->sm_count);
-    p1.x = static_cast<const uint16_t*>(x);
-    p1.amax_row = do_row ? amax_row : nullptr;
-    p1.amax_col = do_col ? amax_col : nullptr;
-    p1.obs = absmax ? ws_obs(ws) : nullptr;
+    // The 1D cast of rows up to kRowPassMaxCols wide encodes rows in the amax pass.
+    const bool row_pass = !w2d && cols <= kRowPassMaxCols;
 
     P2Params<MAXG> p2;
     std::memset(&p2, 0, sizeof p2);
     if ((st = encode_map(&p2.tmap, x, rows, cols)) != NVFP4PT_OK) return st;
-    p2.geo = p1.geo;
-    p2.grp = p1.grp;
+    fill_geometry<MAXG>(p2.geo, p2.grp, rows, cols, off, G, 2 * dev->sm_count, row_pass ? 2 : 1);
     p2.amax_row = amax_row;
     p2.amax_col = amax_col;
     p2.q_row = q_row;
@@ -177,22 +202,55 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
     p2.err = ws_err(ws);
     p2.decay = decay;
     p2.nbuf = absmax ? G : 0;
-    p2.flags = flags;
+    p2.flags = row_pass ? (flags & NVFP4PT_COLWISE) : flags;
 
     ZeroParams z;
     std::memset(&z, 0, sizeof z);
-    if (do_row) { z.ptr[0] = reinterpret_cast<float4*>(amax_row); z.n4[0] = rows / 4; }
+    if (do_row && !row_pass) { z.ptr[0] = reinterpret_cast<float4*>(amax_row); z.n4[0] = rows / 4; }
     if (do_col) { z.ptr[1] = reinterpret_cast<float4*>(amax_col); z.n4[1] = (int64_t)G * cols / 4; }
     if (absmax) { z.ptr[2] = reinterpret_cast<float4*>(ws_obs(ws)); z.n4[2] = pad4(G) / 4; }
     z.err = ws_err(ws);
-
     if (launch_zero(stream, z) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+
     cudaError_t e;
-    if (do_col) e = launch(pass1_amax<MAXG, true>, p1.geo.num_ctas, 0, stream, p1, true);
-    else e = launch(pass1_amax<MAXG, false>, p1.geo.num_ctas, 0, stream, p1, true);
+    if (row_pass) {
+        const RowShape rs = row_shape(cols);
+        RowParams<MAXG> rp;
+        std::memset(&rp, 0, sizeof rp);
+        rp.rows = rows;
+        rp.cols = cols;
+        rp.num_batches = rows / (rs.S * rs.rps);
+        rp.bpr = rs.bpr;
+        rp.tpr = rs.tpr;
+        rp.rps = rs.rps;
+        rp.num_ctas = (int32_t)std::min<int64_t>(rp.num_batches, dev->sm_count);
+        rp.num_groups = G;
+        rp.do_row = do_row;
+        rp.x = static_cast<const uint16_t*>(x);
+        rp.amax_row = do_row ? amax_row : nullptr;
+        rp.q_row = q_row;
+        rp.sf_row = sf_row;
+        rp.amax_col = do_col ? amax_col : nullptr;
+        rp.obs = absmax ? ws_obs(ws) : nullptr;
+        for (int g = 0; g <= G; ++g) rp.row_off[g] = (int32_t)off[g];
+        e = launch_rowpass<MAXG>(rs, rp, stream);
+    } else {
+        P1Params<MAXG> p1;
+        std::memset(&p1, 0, sizeof p1);
+        fill_geometry<MAXG>(p1.geo, p1.grp, rows, cols, off, G, 2 * dev->sm_count, 1);
+        p1.x = static_cast<const uint16_t*>(x);
+        p1.amax_row = do_row ? amax_row : nullptr;
+        p1.amax_col = do_col ? amax_col : nullptr;
+        p1.obs = absmax ? ws_obs(ws) : nullptr;
+        if (do_col) e = launch(pass1_amax<MAXG, true>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
+        else e = launch(pass1_amax<MAXG, false>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
+    }
     if (e != cudaSuccess) return NVFP4PT_ERR_CUDA;
-    if (w2d) e = launch(pass2_encode<MAXG, true>, p2.geo.num_ctas, kSmemPass2, stream, p2, true);
-    else e = launch(pass2_encode<MAXG, false>, p2.geo.num_ctas, kSmemPass2, stream, p2, true);
+    // The encode pass also applies the running-buffer update (its first CTA); with
+    // nothing left to encode it runs that update alone.
+    const int grid2 = p2.flags ? p2.geo.num_ctas : 1;
+    if (w2d) e = launch(pass2_encode<MAXG, true>, grid2, kSmemPass2, stream, p2, true, kThreads);
+    else e = launch(pass2_encode<MAXG, false>, grid2, kSmemPass2, stream, p2, true, kThreads);
     return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 

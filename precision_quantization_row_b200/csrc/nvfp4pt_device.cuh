@@ -37,8 +37,9 @@ struct Geometry {
     int64_t total_tiles;
     int32_t ntc;          // column tiles per band
     int32_t num_groups;
-    int32_t num_ctas;     // CTAs of pass 1 and of pass 2 (same partition)
-    int32_t pad_;
+    int32_t num_ctas;     // CTAs of the launch
+    int32_t interleave;   // CTAs sharing one tile range (1 or 2), each taking every
+                          // interleave-th tile of it
 };
 
 template <int MAXG>
@@ -86,10 +87,26 @@ __device__ __forceinline__ TileInfo tile_info(const Geometry& geo, const Groups<
     return ti;
 }
 
+// Tile range [t0, t1) of a CTA when every CTA owns its own range (interleave 1).
 __device__ __forceinline__ void cta_tile_range(const Geometry& geo, int cta, int64_t& t0, int64_t& t1)
 {
     t0 = (geo.total_tiles * cta) / geo.num_ctas;
     t1 = (geo.total_tiles * (cta + 1)) / geo.num_ctas;
+}
+
+// The encode pass walks its range backwards; with interleave il, CTAs il*k .. il*k+il-1
+// share range k (ranges are cut as for num_ctas / il CTAs) and CTA il*k+j takes tiles
+// t1-1-j, t1-1-j-il, ... . Returns the count n; the i-th tile is last - i * step.
+__device__ __forceinline__ int64_t cta_reverse_tiles(const Geometry& geo, int cta, int64_t& last, int64_t& step)
+{
+    const int il = geo.interleave;
+    const int ranges = geo.num_ctas / il;
+    const int k = cta / il, j = cta - k * il;
+    const int64_t t0 = (geo.total_tiles * k) / ranges;
+    const int64_t t1 = (geo.total_tiles * (k + 1)) / ranges;
+    last = t1 - 1 - j;
+    step = il;
+    return last < t0 ? 0 : (last - t0) / il + 1;
 }
 
 // ----------------------------------------------------- programmatic launch
@@ -125,8 +142,8 @@ __device__ __forceinline__ float absmax_of_pair(uint32_t w)
 // -------------------------------------------------------------- conversions
 
 // Byte of two E2M1 codes, round-to-nearest-even, saturating: `lo` -> bits 0-3,
-// `hi` -> bits 4-7. The hardware conversion puts its first source operand in the
-// high nibble.
+// `hi` -> bits 4-7 (zero-extended to 32 bits). The hardware conversion puts its
+// first source operand in the high nibble.
 __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
 {
     uint32_t r;
@@ -137,20 +154,28 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
     return r;
 }
 
-// Eight products -> one 32-bit word of codes, element i in bits 4i..4i+3.
-__device__ __forceinline__ uint32_t e2m1x8(float y0, float y1, float y2, float y3,
-                                           float y4, float y5, float y6, float y7)
+// Four zero-extended bytes -> one word, b0 in bits 0-7.
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3)
 {
-    uint32_t r;
-    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
-        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
-        : "=r"(r)
-        : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
-    return r;
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// (y0, y1) = (RN(x0 * e), RN(x1 * e)) with one packed two-lane binary32 multiply.
+__device__ __forceinline__ void mul2(float& y0, float& y1, float x0, float x1, float e)
+{
+    unsigned long long a, b, d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(x0), "f"(x1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(e));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(d));
+}
+
+// Codes of the pair (x0, x1) scaled by e: one byte, x0 in the low nibble.
+__device__ __forceinline__ uint32_t code_pair(float x0, float x1, float e)
+{
+    float y0, y1;
+    mul2(y0, y1, x0, x1, e);
+    return e2m1x2(y0, y1);
 }
 
 // Two E4M3 (e4m3fn) codes, round-to-nearest-even, saturating: `lo` -> bits 0-7,
@@ -217,13 +242,22 @@ __device__ __forceinline__ void block_pair_scales(float b0, float b1, float s0, 
     e1 = enc_of(sf01 >> 8, d1, s1);
 }
 
-// Codes of the 8 elements held in 4 bf16 words with one multiplier.
+// Codes of the 8 elements held in 4 bf16 words with one multiplier: one word,
+// element i in bits 4i..4i+3.
 __device__ __forceinline__ uint32_t encode8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float e)
 {
-    return e2m1x8(__fmul_rn(bf16_lo(w0), e), __fmul_rn(bf16_hi(w0), e),
-                  __fmul_rn(bf16_lo(w1), e), __fmul_rn(bf16_hi(w1), e),
-                  __fmul_rn(bf16_lo(w2), e), __fmul_rn(bf16_hi(w2), e),
-                  __fmul_rn(bf16_lo(w3), e), __fmul_rn(bf16_hi(w3), e));
+    return pack4(code_pair(bf16_lo(w0), bf16_hi(w0), e), code_pair(bf16_lo(w1), bf16_hi(w1), e),
+                 code_pair(bf16_lo(w2), bf16_hi(w2), e), code_pair(bf16_lo(w3), bf16_hi(w3), e));
+}
+
+// Codes of one column over 8 consecutive rows, the column being the low (hi=false) or
+// high (hi=true) half of the words x[0..7] (row i in x[i]): one word, row i in bits 4i.
+template <bool HI>
+__device__ __forceinline__ uint32_t encode8_col(const uint32_t* x, float e)
+{
+    auto v = [&](int i) { return HI ? bf16_hi(x[i]) : bf16_lo(x[i]); };
+    return pack4(code_pair(v(0), v(1), e), code_pair(v(2), v(3), e), code_pair(v(4), v(5), e),
+                 code_pair(v(6), v(7), e));
 }
 
 // ---------------------------------------------------------------- memory ops
@@ -234,6 +268,14 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p)
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
+}
+
+// 32 bytes (one 16-element bf16 block) through the read-only path, not kept in L1.
+__device__ __forceinline__ void ldg256_stream(const void* p, uint32_t (&v)[8])
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "l"(p));
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)

@@ -172,7 +172,10 @@ struct P2Params {
     Groups<MAXG> grp;
 };
 
-constexpr int kSmemPass2 = kStages * kStageBytes + 2 * kTile * 4 + kStages * 8 + 1024;
+// staging of one tile's columnwise outputs: codes [128 columns][64 B], scales [128][8 B]
+constexpr int kColCodeBytes = kTile * 64;
+constexpr int kColScaleBytes = kTile * 8;
+constexpr int kSmemPass2 = kStages * kStageBytes + kColCodeBytes + kColScaleBytes + 2 * kTile * 4 + kStages * 8 + 1024;
 
 // Rowwise encode of one half-row (64 columns = 4 blocks) of the tile in `box`.
 // Thread: row r of the tile, half h. W2D: the 16 rows of a band (16 consecutive
@@ -263,22 +266,10 @@ __device__ __forceinline__ void encode_cols(uint32_t box, int p, int hb, float s
         const float ea = b ? e10 : e00;
         const float eb = b ? e11 : e01;
         // column 2p: low halves of rows 16b..16b+15, two per byte (row 2j low nibble)
-        out0[2 * b] = e2m1x8(__fmul_rn(bf16_lo(x[0]), ea), __fmul_rn(bf16_lo(x[1]), ea),
-                             __fmul_rn(bf16_lo(x[2]), ea), __fmul_rn(bf16_lo(x[3]), ea),
-                             __fmul_rn(bf16_lo(x[4]), ea), __fmul_rn(bf16_lo(x[5]), ea),
-                             __fmul_rn(bf16_lo(x[6]), ea), __fmul_rn(bf16_lo(x[7]), ea));
-        out0[2 * b + 1] = e2m1x8(__fmul_rn(bf16_lo(x[8]), ea), __fmul_rn(bf16_lo(x[9]), ea),
-                                 __fmul_rn(bf16_lo(x[10]), ea), __fmul_rn(bf16_lo(x[11]), ea),
-                                 __fmul_rn(bf16_lo(x[12]), ea), __fmul_rn(bf16_lo(x[13]), ea),
-                                 __fmul_rn(bf16_lo(x[14]), ea), __fmul_rn(bf16_lo(x[15]), ea));
-        out1[2 * b] = e2m1x8(__fmul_rn(bf16_hi(x[0]), eb), __fmul_rn(bf16_hi(x[1]), eb),
-                             __fmul_rn(bf16_hi(x[2]), eb), __fmul_rn(bf16_hi(x[3]), eb),
-                             __fmul_rn(bf16_hi(x[4]), eb), __fmul_rn(bf16_hi(x[5]), eb),
-                             __fmul_rn(bf16_hi(x[6]), eb), __fmul_rn(bf16_hi(x[7]), eb));
-        out1[2 * b + 1] = e2m1x8(__fmul_rn(bf16_hi(x[8]), eb), __fmul_rn(bf16_hi(x[9]), eb),
-                                 __fmul_rn(bf16_hi(x[10]), eb), __fmul_rn(bf16_hi(x[11]), eb),
-                                 __fmul_rn(bf16_hi(x[12]), eb), __fmul_rn(bf16_hi(x[13]), eb),
-                                 __fmul_rn(bf16_hi(x[14]), eb), __fmul_rn(bf16_hi(x[15]), eb));
+        out0[2 * b] = encode8_col<false>(x, ea);
+        out0[2 * b + 1] = encode8_col<false>(x + 8, ea);
+        out1[2 * b] = encode8_col<true>(x, eb);
+        out1[2 * b + 1] = encode8_col<true>(x + 8, eb);
     }
 }
 
@@ -287,7 +278,9 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* srow = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+    uint8_t* ccode = smem + kStages * kStageBytes;           // staged column codes
+    uint8_t* cscale = ccode + kColCodeBytes;                  // staged column scales
+    float* srow = reinterpret_cast<float*>(cscale + kColScaleBytes);
     float* scol = srow + kTile;
     uint64_t* bars = reinterpret_cast<uint64_t*>(scol + kTile);
     const uint32_t stage0 = smem_u32(smem);
@@ -298,9 +291,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
     const bool do_row = (p.flags & 1) != 0;
     const bool do_col = !W2D && (p.flags & 2) != 0;
 
-    int64_t t0, t1;
-    cta_tile_range(p.geo, blockIdx.x, t0, t1);
-    const int64_t n = t1 - t0;
+    int64_t last, step;
+    const int64_t n = (do_row || do_col) ? cta_reverse_tiles(p.geo, blockIdx.x, last, step) : 0;
 
     if (tid == 0) {
         prefetch_tensormap(&p.tmap);
@@ -308,9 +300,9 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
         fence_mbar_init();
     }
     __syncthreads();
-    // Tiles go backwards: k-th tile of this CTA is t1 - 1 - k.
+    // Tiles go backwards: the k-th tile of this CTA is last - k * step.
     auto issue = [&](int64_t k) {
-        const TileInfo ti = tile_info(p.geo, p.grp, t1 - 1 - k);
+        const TileInfo ti = tile_info(p.geo, p.grp, last - k * step);
         const int s = (int)(k % kStages);
         const uint32_t bar = bar0 + 8 * s;
         const uint32_t dst = stage0 + s * kStageBytes;
@@ -341,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
         return (do_col && c < ti.nc) ? p.amax_col[(int64_t)ti.g * cols + ti.c0 + c] : 0.0f;
     };
 
-    TileInfo ti = tile_info(p.geo, p.grp, t1 - 1);
+    TileInfo ti = tile_info(p.geo, p.grp, last);
     float a_next = fetch_amax(ti);
     for (int64_t k = 0; k < n; ++k) {
         const int s = (int)(k % kStages);
@@ -351,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
         const float sv = s_enc_of(a_next);
         if (tid < kTile) srow[tid] = sv; else scol[tid - kTile] = sv;
         if (k + 1 < n) {
-            ti = tile_info(p.geo, p.grp, t1 - 2 - k);
+            ti = tile_info(p.geo, p.grp, last - (k + 1) * step);
             a_next = fetch_amax(ti);
         }
         __syncthreads();
@@ -383,27 +375,47 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
                 const int hb = tid >> 6;   // 32-row quarter
                 uint32_t o0[4], o1[4], sf;
                 encode_cols(stage + (pc >> 5) * kBoxBytes, pc, hb, scol[2 * pc], scol[2 * pc + 1], o0, o1, sf);
-                const int nb = min(2, max(0, (cur.nr - 32 * hb) / 16));
-                if (nb > 0) {
-                    const int64_t lrow = cur.r0 - cur.goff;            // first row inside the group
-                    const int64_t gq = cols * (int64_t)cur.goff / 2;    // group's codes start
-                    const int64_t gs = cols * (int64_t)cur.goff / 16;   // group's scales start
-                    const int64_t qstride = cur.grows / 2, sstride = cur.grows / 16;
+                // stage: column c's 64 code bytes hold 16-byte chunk q at slot q ^ ((c >> 1) & 3)
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int64_t col = cur.c0 + 2 * pc + c;
-                        if (2 * pc + c >= cur.nc) break;
-                        const uint32_t* o = c ? o1 : o0;
-                        uint8_t* q = p.q_col + gq + col * qstride + lrow / 2 + 16 * hb;
-                        uint8_t* sfp = p.sf_col + gs + col * sstride + lrow / 16 + 2 * hb;
-                        if (nb == 2) stg16(q, o[0], o[1], o[2], o[3]);
-                        else stg8(q, o[0], o[1]);
-                        stg_bytes(sfp, c ? (sf >> 16) : (sf & 0xFFFFu), nb);
-                    }
+                for (int c = 0; c < 2; ++c) {
+                    const int col = 2 * pc + c;
+                    const uint32_t* o = c ? o1 : o0;
+                    *reinterpret_cast<uint4*>(ccode + col * 64 + 16 * (hb ^ ((col >> 1) & 3))) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint16_t*>(cscale + col * 8 + 2 * hb) = (uint16_t)(c ? (sf >> 16) : sf);
                 }
             }
         }
         const int failed = __syncthreads_or(!ok);
+        if (!failed && do_col) {
+            // coalesced write-back: 4 lanes per column (64 contiguous bytes), then 8 scale bytes
+            const int64_t lrow = cur.r0 - cur.goff;            // first row inside the group
+            const int64_t qstride = cur.grows / 2, sstride = cur.grows / 16;
+            uint8_t* qbase = p.q_col + cols * (int64_t)cur.goff / 2 + lrow / 2;
+            uint8_t* sbase = p.sf_col + cols * (int64_t)cur.goff / 16 + lrow / 16;
+            const int qbytes = cur.nr / 2;                      // code bytes of this tile per column
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int i = tid + kThreads * j;
+                const int col = i >> 2, q = i & 3;
+                if (col < cur.nc && 16 * q < qbytes) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(ccode + col * 64 + 16 * (q ^ ((col >> 1) & 3)));
+                    uint8_t* dst = qbase + (cur.c0 + col) * qstride + 16 * q;
+                    if (16 * q + 16 <= qbytes) stg16(dst, v.x, v.y, v.z, v.w);
+                    else stg8(dst, v.x, v.y);
+                }
+            }
+            if (tid < cur.nc) {
+                const uint2 v = *reinterpret_cast<const uint2*>(cscale + tid * 8);
+                uint8_t* dst = sbase + (cur.c0 + tid) * sstride;
+                const int nb = cur.nr / 16;
+                if (nb == 8 && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0) stg8(dst, v.x, v.y);
+                else {
+                    stg_bytes(dst, v.x, nb < 4 ? nb : 4);
+                    if (nb > 4) stg_bytes(dst + 4, v.y, nb - 4);
+                }
+            }
+        }
         if (failed) {
             // Give up: record the error, let every copy this CTA issued land (bounded),
             // then leave. Stages k .. k+kStages-1 may still have copies in flight.
