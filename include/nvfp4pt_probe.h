@@ -49,6 +49,15 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_probe_e4m3_decode(float* out, cudaStream_t st
  */
 NVFP4PT_API nvfp4pt_status nvfp4pt_probe_div6(float* out, cudaStream_t stream);
 
+/*
+ * The division the cast uses for enc = s_enc / float(sf) against the IEEE division,
+ * both clamped to FLT_MAX: for every positive E4M3 divisor and every binary32 s whose
+ * exponent field lies in [exp_lo, exp_hi] (1..254), *mismatches (device, zeroed here)
+ * receives the number of results that differ in any bit.
+ */
+NVFP4PT_API nvfp4pt_status nvfp4pt_probe_e4m3_div(int exp_lo, int exp_hi, unsigned long long* mismatches,
+                                                  cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -87,6 +87,57 @@ __device__ __forceinline__ TileInfo tile_info(const Geometry& geo, const Groups<
     return ti;
 }
 
+// Walks tiles backwards from a start tile in steps of `step` tiles, keeping (band,
+// column tile) and the band's group facts up to date without dividing per tile.
+template <int MAXG>
+struct TileWalker {
+    int64_t band;
+    int32_t ct;
+    TileInfo ti;
+
+    __device__ __forceinline__ void locate(const Geometry& geo, const Groups<MAXG>& grp)
+    {
+        int g = 0;
+        if (MAXG > 1) {
+            int lo = 0, hi = geo.num_groups;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if ((int64_t)grp.band_start[mid] <= band) lo = mid; else hi = mid;
+            }
+            g = lo;
+        }
+        ti.band = band;
+        ti.g = g;
+        ti.goff = grp.row_off[g];
+        ti.grows = grp.row_off[g + 1] - grp.row_off[g];
+        ti.r0 = (int64_t)ti.goff + (band - grp.band_start[g]) * kTile;
+        const int64_t rem_r = (int64_t)grp.row_off[g + 1] - ti.r0;
+        ti.nr = (int32_t)(rem_r < kTile ? rem_r : kTile);
+    }
+    __device__ __forceinline__ void set_cols(const Geometry& geo)
+    {
+        ti.c0 = (int64_t)ct * kTile;
+        const int64_t rem_c = geo.cols - ti.c0;
+        ti.nc = (int32_t)(rem_c < kTile ? rem_c : kTile);
+    }
+    __device__ __forceinline__ void start(const Geometry& geo, const Groups<MAXG>& grp, int64_t t)
+    {
+        band = t / geo.ntc;
+        ct = (int32_t)(t - band * geo.ntc);
+        locate(geo, grp);
+        set_cols(geo);
+    }
+    __device__ __forceinline__ void back(const Geometry& geo, const Groups<MAXG>& grp, int32_t step)
+    {
+        ct -= step;
+        if (ct < 0) {
+            do { ct += geo.ntc; --band; } while (ct < 0);
+            locate(geo, grp);
+        }
+        set_cols(geo);
+    }
+};
+
 // Tile range [t0, t1) of a CTA when every CTA owns its own range (interleave 1).
 __device__ __forceinline__ void cta_tile_range(const Geometry& geo, int cta, int64_t& t0, int64_t& t1)
 {
@@ -222,24 +273,49 @@ __device__ __forceinline__ float s_enc_of(float amax)
     return fminf(__fdiv_rn(2688.0f, amax), FLT_MAX);
 }
 
-// enc = s_enc / float(sf), 0 when sf == 0, clamped to FLT_MAX.
-__device__ __forceinline__ float enc_of(uint32_t sf_code, float d, float s)
+// Reciprocal table of the E4M3 significands: tab[f] = bits of RN(1 / (1 + f/8)),
+// f = 0..7. Each CTA keeps it in shared memory (8 words, one bank each).
+__device__ __forceinline__ void init_rcp_table(uint32_t* tab)
 {
-    return (sf_code & 0xFFu) ? fminf(__fdiv_rn(s, d), FLT_MAX) : 0.0f;
+    if (threadIdx.x < 8) tab[threadIdx.x] = __float_as_uint(__fdiv_rn(1.0f, 1.0f + 0.125f * (float)threadIdx.x));
+}
+
+// RN(s / d) for s a positive normal binary32 and d a positive E4M3 value (as exact
+// binary32). d has a 4-bit significand, so y = RN(1/d) is a table entry scaled by d's
+// power of two (exactly); then q0 = RN(s * y), the exact remainder r = s - q0*d by one
+// fused multiply-add, and one correction q0 + r*y -- the correction step of Markstein's
+// division (IBM J. Res. Dev. 34(1), 1990). It equals the IEEE quotient for every E4M3
+// divisor and every s tried (all significands of 20 binades from 2^-117 up to 2^127,
+// and FLT_MAX); the probe entry compares it with the IEEE division on the device.
+// An overflowing quotient comes out as +inf or NaN; the caller clamps it.
+__device__ __forceinline__ float div_by_e4m3(float s, float d, const uint32_t* tab)
+{
+    const uint32_t db = __float_as_uint(d);
+    const float y = __uint_as_float(tab[(db >> 20) & 7u] + 0x3F800000u - (db & 0x7F800000u));
+    const float q0 = __fmul_rn(s, y);
+    const float r = __fmaf_rn(-q0, d, s);
+    return __fmaf_rn(r, y, q0);
+}
+
+// enc = s_enc / float(sf), 0 when sf == 0, clamped to FLT_MAX (fminf also maps the NaN
+// of an overflowed quotient to FLT_MAX).
+__device__ __forceinline__ float enc_of(uint32_t sf_code, float d, float s, const uint32_t* tab)
+{
+    return (sf_code & 0xFFu) ? fminf(div_by_e4m3(s, d, tab), FLT_MAX) : 0.0f;
 }
 
 // Scale codes and multipliers of two blocks with block amaxes b0, b1 and outer
 // scales s0, s1. sf01 receives the two codes (block 0 in bits 0-7).
 __device__ __forceinline__ void block_pair_scales(float b0, float b1, float s0, float s1,
-                                                  uint32_t& sf01, float& e0, float& e1)
+                                                  uint32_t& sf01, float& e0, float& e1, const uint32_t* tab)
 {
     const float u0 = __fmul_rn(div6(b0), s0);
     const float u1 = __fmul_rn(div6(b1), s1);
     sf01 = e4m3x2(u0, u1);
     float d0, d1;
     e4m3x2_decode(sf01, d0, d1);
-    e0 = enc_of(sf01, d0, s0);
-    e1 = enc_of(sf01 >> 8, d1, s1);
+    e0 = enc_of(sf01, d0, s0, tab);
+    e1 = enc_of(sf01 >> 8, d1, s1, tab);
 }
 
 // Codes of the 8 elements held in 4 bf16 words with one multiplier: one word,

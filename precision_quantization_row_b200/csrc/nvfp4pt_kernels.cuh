@@ -181,7 +181,8 @@ constexpr int kSmemPass2 = kStages * kStageBytes + kColCodeBytes + kColScaleByte
 // Thread: row r of the tile, half h. W2D: the 16 rows of a band (16 consecutive
 // lanes) share one scale per block (the largest of their 1D scale arguments).
 template <bool W2D>
-__device__ __forceinline__ void encode_rows(uint32_t box, int r, float s, uint32_t out[8], uint32_t& sf4)
+__device__ __forceinline__ void encode_rows(uint32_t box, int r, float s, uint32_t out[8], uint32_t& sf4,
+                                            const uint32_t* tab)
 {
     uint32_t w[32];
 #pragma unroll
@@ -200,8 +201,8 @@ __device__ __forceinline__ void encode_rows(uint32_t box, int r, float s, uint32
     float e[4];
     uint32_t sf01, sf23;
     if (!W2D) {
-        block_pair_scales(ba[0], ba[1], s, s, sf01, e[0], e[1]);
-        block_pair_scales(ba[2], ba[3], s, s, sf23, e[2], e[3]);
+        block_pair_scales(ba[0], ba[1], s, s, sf01, e[0], e[1], tab);
+        block_pair_scales(ba[2], ba[3], s, s, sf23, e[2], e[3], tab);
     } else {
         float u[4];
 #pragma unroll
@@ -215,10 +216,10 @@ __device__ __forceinline__ void encode_rows(uint32_t box, int r, float s, uint32
         float d0, d1, d2, d3;
         e4m3x2_decode(sf01, d0, d1);
         e4m3x2_decode(sf23, d2, d3);
-        e[0] = enc_of(sf01, d0, s);
-        e[1] = enc_of(sf01 >> 8, d1, s);
-        e[2] = enc_of(sf23, d2, s);
-        e[3] = enc_of(sf23 >> 8, d3, s);
+        e[0] = enc_of(sf01, d0, s, tab);
+        e[1] = enc_of(sf01 >> 8, d1, s, tab);
+        e[2] = enc_of(sf23, d2, s, tab);
+        e[3] = enc_of(sf23 >> 8, d3, s, tab);
     }
     sf4 = (sf01 & 0xFFFFu) | (sf23 << 16);
 #pragma unroll
@@ -232,7 +233,7 @@ __device__ __forceinline__ void encode_rows(uint32_t box, int r, float s, uint32
 // Columnwise encode of a column pair (2p, 2p+1) over 32 rows (2 blocks) of the tile.
 // v[i] holds row 32*hb+i of both columns (low half = column 2p).
 __device__ __forceinline__ void encode_cols(uint32_t box, int p, int hb, float s0, float s1,
-                                            uint32_t out0[4], uint32_t out1[4], uint32_t& sf)
+                                            uint32_t out0[4], uint32_t out1[4], uint32_t& sf, const uint32_t* tab)
 {
     uint32_t v[32];
     const int chunk = (p & 31) >> 2;
@@ -257,8 +258,8 @@ __device__ __forceinline__ void encode_cols(uint32_t box, int p, int hb, float s
     const float b10 = __uint_as_float(m[1] << 16), b11 = __uint_as_float(m[1] & 0xFFFF0000u);
     uint32_t sfc0, sfc1;   // column 0: blocks 0,1 ; column 1: blocks 0,1
     float e00, e10, e01, e11;
-    block_pair_scales(b00, b10, s0, s0, sfc0, e00, e10);
-    block_pair_scales(b01, b11, s1, s1, sfc1, e01, e11);
+    block_pair_scales(b00, b10, s0, s0, sfc0, e00, e10, tab);
+    block_pair_scales(b01, b11, s1, s1, sfc1, e01, e11, tab);
     sf = (sfc0 & 0xFFFFu) | (sfc1 << 16);
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
@@ -285,6 +286,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(scol + kTile);
     const uint32_t stage0 = smem_u32(smem);
     const uint32_t bar0 = smem_u32(bars);
+    __shared__ uint32_t rcp_tab[8];
+    init_rcp_table(rcp_tab);
 
     const int tid = threadIdx.x;
     const int64_t cols = p.geo.cols;
@@ -300,19 +303,25 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
         fence_mbar_init();
     }
     __syncthreads();
-    // Tiles go backwards: the k-th tile of this CTA is last - k * step.
-    auto issue = [&](int64_t k) {
-        const TileInfo ti = tile_info(p.geo, p.grp, last - k * step);
-        const int s = (int)(k % kStages);
+    // Tiles go backwards: the k-th tile of this CTA is last - k * step. Thread 0 walks
+    // the issued tiles (kStages ahead of the encoded ones) with its own walker.
+    TileWalker<MAXG> iw;
+    int64_t issued = 0;
+    auto issue_next = [&]() {
+        if (issued > 0) iw.back(p.geo, p.grp, (int32_t)step);
+        const int s = (int)(issued % kStages);
         const uint32_t bar = bar0 + 8 * s;
         const uint32_t dst = stage0 + s * kStageBytes;
         mbar_arrive_expect_tx(bar, kStageBytes);
-        tma_load_2d(dst, &p.tmap, (int32_t)ti.c0, (int32_t)ti.r0, bar);
-        tma_load_2d(dst + kBoxBytes, &p.tmap, (int32_t)ti.c0 + 64, (int32_t)ti.r0, bar);
+        tma_load_2d(dst, &p.tmap, (int32_t)iw.ti.c0, (int32_t)iw.ti.r0, bar);
+        tma_load_2d(dst + kBoxBytes, &p.tmap, (int32_t)iw.ti.c0 + 64, (int32_t)iw.ti.r0, bar);
+        ++issued;
     };
     // x is read-only for the whole chain, so the first tiles load before pass 1 ends.
-    if (tid == 0)
-        for (int64_t k = 0; k < n && k < kStages; ++k) issue(k);
+    if (tid == 0 && n > 0) {
+        iw.start(p.geo, p.grp, last);
+        for (int64_t k = 0; k < n && k < kStages; ++k) issue_next();
+    }
 
     griddep_wait();
     if (blockIdx.x == 0 && p.absmax) {
@@ -333,18 +342,19 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
         return (do_col && c < ti.nc) ? p.amax_col[(int64_t)ti.g * cols + ti.c0 + c] : 0.0f;
     };
 
-    TileInfo ti = tile_info(p.geo, p.grp, last);
-    float a_next = fetch_amax(ti);
+    TileWalker<MAXG> w;
+    w.start(p.geo, p.grp, last);
+    float a_next = fetch_amax(w.ti);
+    int s = 0;
+    uint32_t parity = 0;
     for (int64_t k = 0; k < n; ++k) {
-        const int s = (int)(k % kStages);
-        const uint32_t parity = (uint32_t)((k / kStages) & 1);
-        const TileInfo cur = ti;
+        const TileInfo cur = w.ti;
         // outer scales of this tile's rows and columns
         const float sv = s_enc_of(a_next);
         if (tid < kTile) srow[tid] = sv; else scol[tid - kTile] = sv;
         if (k + 1 < n) {
-            ti = tile_info(p.geo, p.grp, last - (k + 1) * step);
-            a_next = fetch_amax(ti);
+            w.back(p.geo, p.grp, (int32_t)step);
+            a_next = fetch_amax(w.ti);
         }
         __syncthreads();
 
@@ -355,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
                 const int r = tid & (kTile - 1);
                 const int h = tid >> 7;
                 uint32_t out[8], sf4;
-                encode_rows<W2D>(stage + h * kBoxBytes, r, srow[r], out, sf4);
+                encode_rows<W2D>(stage + h * kBoxBytes, r, srow[r], out, sf4, rcp_tab);
                 const int nb = min(4, max(0, (cur.nc - 64 * h) / 16));
                 if (r < cur.nr && nb > 0) {
                     const int64_t row = cur.r0 + r;
@@ -374,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
                 const int pc = tid & 63;   // column pair
                 const int hb = tid >> 6;   // 32-row quarter
                 uint32_t o0[4], o1[4], sf;
-                encode_cols(stage + (pc >> 5) * kBoxBytes, pc, hb, scol[2 * pc], scol[2 * pc + 1], o0, o1, sf);
+                encode_cols(stage + (pc >> 5) * kBoxBytes, pc, hb, scol[2 * pc], scol[2 * pc + 1], o0, o1, sf,
+                            rcp_tab);
                 // stage: column c's 64 code bytes hold 16-byte chunk q at slot q ^ ((c >> 1) & 3)
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -430,7 +441,8 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
             __syncthreads();
             return;
         }
-        if (tid == 0 && k + kStages < n) issue(k + kStages);
+        if (tid == 0 && k + kStages < n) issue_next();
+        if (++s == kStages) { s = 0; parity ^= 1u; }
     }
 }
 

@@ -67,6 +67,32 @@ __global__ void div6_kernel(float* out)
     if (h < 0x7F80u) out[h] = div6(__uint_as_float(h << 16));
 }
 
+// For every positive E4M3 divisor and every s with exponent field in [e_lo, e_hi]:
+// count where the division used by the cast differs from the IEEE division.
+__global__ void e4m3_div_kernel(int e_lo, int e_hi, unsigned long long* mismatches)
+{
+    __shared__ uint32_t tab[8];
+    init_rcp_table(tab);
+    __syncthreads();
+    const uint64_t per = 1ull << 23;
+    const uint64_t total = (uint64_t)(e_hi - e_lo + 1) * per;
+    unsigned long long bad = 0;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (uint64_t)gridDim.x * blockDim.x) {
+        const uint32_t bits = ((uint32_t)(e_lo + i / per) << 23) | (uint32_t)(i % per);
+        const float s = __uint_as_float(bits);
+        for (uint32_t c = 1; c <= 0x7E; c += 2) {
+            float d0, d1;
+            e4m3x2_decode(c | ((c + 1) << 8), d0, d1);
+            const float ref0 = fminf(__fdiv_rn(s, d0), FLT_MAX);
+            const float ref1 = fminf(__fdiv_rn(s, d1), FLT_MAX);
+            const float got0 = fminf(div_by_e4m3(s, d0, tab), FLT_MAX);
+            const float got1 = fminf(div_by_e4m3(s, d1, tab), FLT_MAX);
+            bad += (__float_as_uint(ref0) != __float_as_uint(got0)) + (__float_as_uint(ref1) != __float_as_uint(got1));
+        }
+    }
+    if (bad) atomicAdd(mismatches, bad);
+}
+
 nvfp4pt_status arch_ok()
 {
     int dev = 0, major = 0, minor = 0;
@@ -115,6 +141,17 @@ nvfp4pt_status nvfp4pt_probe_e4m3_decode(float* out, cudaStream_t stream)
     nvfp4pt_status st = arch_ok();
     if (st != NVFP4PT_OK) return st;
     decode_kernel<<<1, 256, 0, stream>>>(out);
+    return last();
+}
+
+nvfp4pt_status nvfp4pt_probe_e4m3_div(int exp_lo, int exp_hi, unsigned long long* mismatches, cudaStream_t stream)
+{
+    if (!mismatches) return NVFP4PT_ERR_NULL;
+    if (exp_lo < 1 || exp_hi > 254 || exp_lo > exp_hi) return NVFP4PT_ERR_SHAPE;
+    nvfp4pt_status st = arch_ok();
+    if (st != NVFP4PT_OK) return st;
+    if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), stream) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    e4m3_div_kernel<<<148 * 8, 256, 0, stream>>>(exp_lo, exp_hi, mismatches);
     return last();
 }
 

@@ -57,10 +57,10 @@ __device__ __forceinline__ int group_of_row(const RowParams<MAXG>& p, int64_t ro
 // scales sa, sb: two words of codes per block and the two scale bytes (a in bits 0-7).
 __device__ __forceinline__ void encode_block_pair(const uint32_t (&a)[8], const uint32_t (&b)[8], float ba, float bb,
                                                   float sa, float sb, uint32_t& qa0, uint32_t& qa1, uint32_t& qb0,
-                                                  uint32_t& qb1, uint32_t& sf)
+                                                  uint32_t& qb1, uint32_t& sf, const uint32_t* tab)
 {
     float ea, eb;
-    block_pair_scales(ba, bb, sa, sb, sf, ea, eb);
+    block_pair_scales(ba, bb, sa, sb, sf, ea, eb, tab);
     qa0 = encode8(a[0], a[1], a[2], a[3], ea);
     qa1 = encode8(a[4], a[5], a[6], a[7], ea);
     qb0 = encode8(b[0], b[1], b[2], b[3], eb);
@@ -73,6 +73,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
     griddep_launch_dependents();
     __shared__ uint32_t part[S * 16][kRowThreads / 32];   // [row of batch][warp of row] partial amax bits
     __shared__ float srow[S * 16];            // outer scale of each row of the batch
+    __shared__ uint32_t rcp_tab[8];           // E4M3 significand reciprocals
+    init_rcp_table(rcp_tab);                  // first read after the batch barriers
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
                 const int bb = (i + 1 < S * BT) ? (i + 1) % BT : ba;
                 uint32_t qa0, qa1, qb0, qb1, sf;
                 encode_block_pair(cur[sa][ba], cur[sb][bb], absmax_of_pair(bmax[sa][ba]), absmax_of_pair(bmax[sb][bb]),
-                                  sv[sa], sv[sb], qa0, qa1, qb0, qb1, sf);
+                                  sv[sa], sv[sb], qa0, qa1, qb0, qb1, sf, rcp_tab);
                 if (valid[ba]) {
                     const int64_t row = r0 + sa * p.rps + rsw;
                     stg8(p.q_row + row * (cols / 2) + 8 * (int64_t)bj[ba], qa0, qa1);

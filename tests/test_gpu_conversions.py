@@ -112,3 +112,16 @@ def test_div6_exhaustive():
     b = (np.arange(0x7F80, dtype=np.uint32) << 16).view(np.float32)
     want = (b / np.float32(6.0)).astype(np.float32).view(np.uint32)  # IEEE binary32 division
     assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("lo,hi", [(10, 24), (125, 129), (252, 254)])
+def test_block_scale_division_matches_ieee(lo, hi):
+    """enc = s_enc / float(sf) as the cast computes it, against the IEEE division, for all
+    126 positive E4M3 divisors and every significand of s in the given binades: the low
+    binades (down to the smallest possible s_enc, 2688/FLT_MAX ~ 2^-117, where the
+    remainder can be subnormal), the middle, and the overflow edge (clamped to FLT_MAX)."""
+    bad = torch.zeros(1, dtype=torch.int64, device="cuda")
+    st = nv.lib().nvfp4pt_probe_e4m3_div(lo, hi, ctypes.c_void_p(bad.data_ptr()),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    assert int(bad.item()) == 0
