@@ -156,6 +156,31 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_update_absmax(float* absmax_buf, const float*
                                      float decay, cudaStream_t stream);
 
 /*
+ * nvfp4pt_quantize_grouped_noalloc -- nvfp4pt_quantize_grouped for callers that cannot
+ * allocate device memory (no counterpart in the cast's description: it exists for
+ * callers whose code must not allocate -- inside an allocator or memory-pool callback,
+ * under a fixed memory budget, or with no workspace to hand over).
+ *
+ * Same arguments and results as nvfp4pt_quantize_grouped, without the workspace: the
+ * scratch lives in a static device array of NVFP4PT_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads the library holds until the process exits. The
+ * call allocates nothing (no cudaMalloc, no allocating library routine).
+ *   - num_groups above NVFP4PT_NOALLOC_MAX_GROUPS (what the array holds) returns
+ *     NVFP4PT_ERR_GROUPS before anything is launched.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call shares the array and clears what it accumulates at its start; calls
+ *     that overlap on the GPU (different streams, or different host threads) race on it.
+ */
+#define NVFP4PT_NOALLOC_SCRATCH_BYTES 1024
+#define NVFP4PT_NOALLOC_MAX_GROUPS 252
+NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_grouped_noalloc(const void* x_bf16, int64_t rows, int64_t cols,
+                                        const int64_t* offsets_host, int num_groups, int flags,
+                                        uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                        uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                        float* absmax_bufs, float decay, cudaStream_t stream);
+
+/*
  * nvfp4pt_workspace_error -- read the device error word the last call on this
  * workspace left (0 = none). Synchronises `stream`. A nonzero word means a kernel
  * gave up a bounded wait (a TMA copy that never arrived) and skipped the rest of its

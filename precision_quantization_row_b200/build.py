@@ -14,8 +14,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libnvfp4pt.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("nvfp4pt_api.cu", "nvfp4pt_probe.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh")] + \
+SOURCES = [os.path.join(CSRC, f) for f in ("nvfp4pt_api.cu", "nvfp4pt_probe.cu", "nvfp4pt_noalloc.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh",
+                                                  "nvfp4pt_rowpass.cuh")] + \
     [os.path.join(INCLUDE, f) for f in ("nvfp4pt.h", "nvfp4pt_probe.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
