@@ -58,6 +58,17 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_probe_div6(float* out, cudaStream_t stream);
 NVFP4PT_API nvfp4pt_status nvfp4pt_probe_e4m3_div(int exp_lo, int exp_hi, unsigned long long* mismatches,
                                                   cudaStream_t stream);
 
+/*
+ * The block-scale step (sf = E4M3(RN(b/6) * s), enc = s / float(sf)) as the cast's
+ * packed two-lane form computes it, against its scalar form, which the tests pin to
+ * the oracle: for every non-negative finite bf16 block amax b and every `stride`-th
+ * significand of s in each binade whose exponent field lies in [exp_lo, exp_hi]
+ * (1..254), plus s = FLT_MAX and s = 1, *mismatches (device, zeroed here) receives
+ * the number of scale codes or multipliers that differ in any bit. stride >= 1.
+ */
+NVFP4PT_API nvfp4pt_status nvfp4pt_probe_pair_scales(int exp_lo, int exp_hi, unsigned int stride,
+                                                     unsigned long long* mismatches, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,7 +34,7 @@ EXPORTS = (
     "nvfp4pt_status_string", "nvfp4pt_workspace_bytes", "nvfp4pt_quantize", "nvfp4pt_quantize_grouped",
     "nvfp4pt_quantize_weight_2d", "nvfp4pt_update_absmax", "nvfp4pt_workspace_error",
     "nvfp4pt_probe_transitions", "nvfp4pt_probe_pairs", "nvfp4pt_probe_e4m3_decode", "nvfp4pt_probe_div6",
-    "nvfp4pt_probe_e4m3_div", "nvfp4pt_quantize_grouped_noalloc",
+    "nvfp4pt_probe_e4m3_div", "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_probe_pair_scales",
 )
 
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_probe_div6.argtypes = [P, P]
         L.nvfp4pt_probe_e4m3_div.argtypes = [I, I, P, P]
         L.nvfp4pt_quantize_grouped_noalloc.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, F, P]
+        L.nvfp4pt_probe_pair_scales.argtypes = [I, I, ctypes.c_uint32, P, P]
         for name in EXPORTS[2:]:
             getattr(L, name).restype = I
         _lib = L

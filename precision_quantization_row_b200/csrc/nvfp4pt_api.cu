@@ -10,6 +10,7 @@
 #include "nvfp4pt.h"
 #include "nvfp4pt_kernels.cuh"
 #include "nvfp4pt_rowpass.cuh"
+#include "nvfp4pt_colpass.cuh"
 
 using namespace nvfp4pt;
 
@@ -51,6 +52,11 @@ nvfp4pt_status device_state(DeviceState** out)
             for (const void* f : encoders) {
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPass2) != cudaSuccess ||
                     cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+                    return NVFP4PT_ERR_CUDA;
+            }
+            const void* colpasses[] = {(const void*)colpass<1>, (const void*)colpass<kMaxGroups>};
+            for (const void* f : colpasses) {
+                if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColPass) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
             }
             if (!g_encode) {
@@ -187,23 +193,6 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
     // The 1D cast of rows up to kRowPassMaxCols wide encodes rows in the amax pass.
     const bool row_pass = !w2d && cols <= kRowPassMaxCols;
 
-    P2Params<MAXG> p2;
-    std::memset(&p2, 0, sizeof p2);
-    if ((st = encode_map(&p2.tmap, x, rows, cols)) != NVFP4PT_OK) return st;
-    fill_geometry<MAXG>(p2.geo, p2.grp, rows, cols, off, G, 2 * dev->sm_count, row_pass ? 2 : 1);
-    p2.amax_row = amax_row;
-    p2.amax_col = amax_col;
-    p2.q_row = q_row;
-    p2.sf_row = sf_row;
-    p2.q_col = q_col;
-    p2.sf_col = sf_col;
-    p2.absmax = absmax;
-    p2.obs = ws_obs(ws);
-    p2.err = ws_err(ws);
-    p2.decay = decay;
-    p2.nbuf = absmax ? G : 0;
-    p2.flags = row_pass ? (flags & NVFP4PT_COLWISE) : flags;
-
     ZeroParams z;
     std::memset(&z, 0, sizeof z);
     if (do_row && !row_pass) { z.ptr[0] = reinterpret_cast<float4*>(amax_row); z.n4[0] = rows / 4; }
@@ -226,6 +215,7 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         rp.num_ctas = (int32_t)std::min<int64_t>(rp.num_batches, dev->sm_count);
         rp.num_groups = G;
         rp.do_row = do_row;
+        rp.strided = G == 1;
         rp.x = static_cast<const uint16_t*>(x);
         rp.amax_row = do_row ? amax_row : nullptr;
         rp.q_row = q_row;
@@ -233,24 +223,72 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         rp.amax_col = do_col ? amax_col : nullptr;
         rp.obs = absmax ? ws_obs(ws) : nullptr;
         for (int g = 0; g <= G; ++g) rp.row_off[g] = (int32_t)off[g];
-        e = launch_rowpass<MAXG>(rs, rp, stream);
-    } else {
-        P1Params<MAXG> p1;
-        std::memset(&p1, 0, sizeof p1);
-        fill_geometry<MAXG>(p1.geo, p1.grp, rows, cols, off, G, 2 * dev->sm_count, 1);
-        p1.x = static_cast<const uint16_t*>(x);
-        p1.amax_row = do_row ? amax_row : nullptr;
-        p1.amax_col = do_col ? amax_col : nullptr;
-        p1.obs = absmax ? ws_obs(ws) : nullptr;
-        if (do_col) e = launch(pass1_amax<MAXG, true>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
-        else e = launch(pass1_amax<MAXG, false>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
+        if ((e = launch_rowpass<MAXG>(rs, rp, stream)) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+
+        // Column pass: 256-row tasks per group (the last one ragged) x 32-column strips.
+        // With nothing to encode it runs the running-buffer update alone (one CTA).
+        ColParams<MAXG> cp;
+        std::memset(&cp, 0, sizeof cp);
+        int32_t tasks = 0;
+        for (int g = 0; g < G; ++g) {
+            cp.row_off[g] = (int32_t)off[g];
+            cp.task_off[g] = tasks;
+            tasks += (int32_t)((off[g + 1] - off[g] + kTaskRows - 1) / kTaskRows);
+        }
+        cp.row_off[G] = (int32_t)off[G];
+        cp.task_off[G] = tasks;
+        cp.cols = cols;
+        cp.strips = (int32_t)((cols + kTaskCols - 1) / kTaskCols);
+        cp.num_tasks = do_col ? (int64_t)tasks * cp.strips : 0;
+        cp.num_ctas = (int32_t)std::max<int64_t>(
+            1, std::min<int64_t>(dev->sm_count, (cp.num_tasks + kColWarps - 1) / kColWarps));
+        cp.num_groups = G;
+        cp.nbuf = absmax ? G : 0;
+        cp.decay = decay;
+        cp.q_col_32 = (reinterpret_cast<uintptr_t>(q_col) & 31u) == 0;
+        cp.strided = G == 1;
+        const int64_t wstride = cp.strided ? (int64_t)cp.num_ctas * kColWarps : kColWarps;
+        cp.back_rt = (int32_t)(wstride / cp.strips);
+        cp.back_strip = (int32_t)(wstride % cp.strips);
+        cp.x = static_cast<const uint16_t*>(x);
+        cp.amax_col = amax_col;
+        cp.q_col = q_col;
+        cp.sf_col = sf_col;
+        cp.absmax = absmax;
+        cp.obs = ws_obs(ws);
+        e = launch(colpass<MAXG>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
+        return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
     }
+
+    P2Params<MAXG> p2;
+    std::memset(&p2, 0, sizeof p2);
+    if ((st = encode_map(&p2.tmap, x, rows, cols)) != NVFP4PT_OK) return st;
+    fill_geometry<MAXG>(p2.geo, p2.grp, rows, cols, off, G, 2 * dev->sm_count, 1);
+    p2.amax_row = amax_row;
+    p2.amax_col = amax_col;
+    p2.q_row = q_row;
+    p2.sf_row = sf_row;
+    p2.q_col = q_col;
+    p2.sf_col = sf_col;
+    p2.absmax = absmax;
+    p2.obs = ws_obs(ws);
+    p2.err = ws_err(ws);
+    p2.decay = decay;
+    p2.nbuf = absmax ? G : 0;
+    p2.flags = flags;
+
+    P1Params<MAXG> p1;
+    std::memset(&p1, 0, sizeof p1);
+    fill_geometry<MAXG>(p1.geo, p1.grp, rows, cols, off, G, 2 * dev->sm_count, 1);
+    p1.x = static_cast<const uint16_t*>(x);
+    p1.amax_row = do_row ? amax_row : nullptr;
+    p1.amax_col = do_col ? amax_col : nullptr;
+    p1.obs = absmax ? ws_obs(ws) : nullptr;
+    if (do_col) e = launch(pass1_amax<MAXG, true>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
+    else e = launch(pass1_amax<MAXG, false>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
     if (e != cudaSuccess) return NVFP4PT_ERR_CUDA;
-    // The encode pass also applies the running-buffer update (its first CTA); with
-    // nothing left to encode it runs that update alone.
-    const int grid2 = p2.flags ? p2.geo.num_ctas : 1;
-    if (w2d) e = launch(pass2_encode<MAXG, true>, grid2, kSmemPass2, stream, p2, true, kThreads);
-    else e = launch(pass2_encode<MAXG, false>, grid2, kSmemPass2, stream, p2, true, kThreads);
+    if (w2d) e = launch(pass2_encode<MAXG, true>, p2.geo.num_ctas, kSmemPass2, stream, p2, true, kThreads);
+    else e = launch(pass2_encode<MAXG, false>, p2.geo.num_ctas, kSmemPass2, stream, p2, true, kThreads);
     return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 

@@ -1,0 +1,335 @@
+// Column pass of the NVFP4 per-token cast (sm_100a): the columnwise encode (codes and
+// E4M3 scales of X^T) once the row pass has left the per-column amax of every token
+// group in amax_col. It reads x once more, straight into registers: no shared-memory
+// tiles of x, no block barriers in the loop.
+//
+// Layout of the work: a "task" is up to 256 rows x 32 columns of one token group,
+// given to one warp and taken in "steps" of 64 rows. In a step, lane l = 4q + s holds
+// the 16 rows 16s..16s+15 of the step's columns 4q..4q+3 (one 8-byte load per row),
+// encodes its four 16-row blocks and parks codes and scales in the warp's staging
+// area. After the task's last step the warp writes the task's columns: up to 128 code
+// bytes per column (one whole L2 line), eight lanes to a line so that each store
+// instruction covers four lines, and 16 scale bytes per column. Whole lines matter:
+// column outputs are strided by the group's row count, and lines written a sector at
+// a time, far apart in time, go back to DRAM a sector at a time.
+//
+// Tasks are numbered row-task-major over all groups and walked backwards, each warp
+// prefetching the next step's rows into a second register buffer. With one token group the grid's warps take tasks
+// T-1-w, T-1-w-W, ... (W warps in all): the grid sweeps x from the bottom up as one
+// front and starts on the rows that the row pass, sweeping downwards, read last and
+// left in L2. With several groups CTA c owns a contiguous run of tasks, warp w taking
+// every 16th from its end, which lines up with the contiguous runs of the row pass.
+#pragma once
+
+#include "nvfp4pt_device.cuh"
+
+namespace nvfp4pt {
+
+constexpr int kColThreads = 512;   // one CTA per SM: 128 registers per thread
+constexpr int kColWarps = kColThreads / 32;
+constexpr int kStepRows = 64;      // rows of a step: four 16-row blocks
+constexpr int kTaskRows = 256;     // rows of a task: up to four steps
+constexpr int kTaskCols = 32;      // columns of a task: 8 quads x 4
+constexpr int kColStageBytes = kTaskCols * (128 + 16);      // per warp: codes, scales
+constexpr int kSmemColPass = kColWarps * kColStageBytes;    // dynamic shared memory
+
+template <int MAXG>
+struct ColParams {
+    int64_t cols;
+    int64_t num_tasks;   // row tasks x strips
+    int32_t strips;      // ceil(cols / 32)
+    int32_t num_ctas;
+    int32_t num_groups;
+    int32_t nbuf;        // running buffers to update (0: none)
+    float decay;
+    int32_t q_col_32;    // q_col is 32-byte aligned: full column segments go in one store
+    int32_t strided;     // one front over the whole grid (else a contiguous run per CTA)
+    int32_t back_rt;     // a warp's next task is wstride tasks back:
+    int32_t back_strip;  //   wstride = back_rt * strips + back_strip, back_strip < strips
+    const uint16_t* x;
+    const float* amax_col;   // [G, cols], final when the row pass has ended
+    uint8_t* q_col;
+    uint8_t* sf_col;
+    float* absmax;           // [nbuf] running amax buffers, or null
+    const float* obs;        // [G] amax observed by the row pass
+    int32_t row_off[MAXG + 1];    // first row of each group
+    int32_t task_off[MAXG + 1];   // first row task of each group
+};
+
+// 8 bytes through the read-only path, not kept in L1.
+__device__ __forceinline__ uint2 ldg64_stream(const void* p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+// Codes of 8 consecutive rows of one column with one multiplier; the column is the
+// low (HI = false) or high half of the bf16 words v[r0 .. r0+7][w]. Row i -> bits 4i.
+template <bool HI>
+__device__ __forceinline__ uint32_t encode8_strided(const uint32_t (&v)[16][2], int r0, int w, float e)
+{
+    auto val = [&](int i) { return HI ? bf16_hi(v[r0 + i][w]) : bf16_lo(v[r0 + i][w]); };
+    float y[8];
+    mul2(y[0], y[1], val(0), val(1), e);
+    mul2(y[2], y[3], val(2), val(3), e);
+    mul2(y[4], y[5], val(4), val(5), e);
+    mul2(y[6], y[7], val(6), val(7), e);
+    return e2m1x8_packed(y);
+}
+
+// Where a task sits: its group, first row, row count and first column.
+struct ColTask {
+    int32_t row0;
+    int32_t goff;
+    int32_t grows;
+    int32_t c0;
+    int32_t nrows;    // 16..256, a multiple of 16
+};
+
+// Staging slot of 8-byte chunk k (16 rows) of column c: 16-byte chunk (k >> 1) ^ g(c)
+// of the column's 128-byte row. g keeps both the lanes' 8-byte stores of a step and
+// the column reads of the write-out free of bank conflicts.
+__device__ __forceinline__ int stage_off(int c, int k)
+{
+    const int g = (c & 7) ^ ((c >> 2) & 6);
+    return c * 128 + 16 * ((k >> 1) ^ g) + 8 * (k & 1);
+}
+
+template <int MAXG>
+__device__ __forceinline__ int group_of_task(const ColParams<MAXG>& p, int rt)
+{
+    if (MAXG == 1) return 0;
+    int lo = 0, hi = p.num_groups;  // task_off[lo] <= rt < task_off[hi]; empty groups skipped
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (p.task_off[mid] <= rt) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+template <int MAXG>
+__global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant__ ColParams<MAXG> p)
+{
+    // per warp: codes [column][16 chunks of 8 bytes] (swizzled), then scales [column][16]
+    extern __shared__ __align__(16) uint8_t col_stage[];
+    __shared__ uint32_t rcp_tab[8];
+    init_rcp_table(rcp_tab);
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int quad = lane >> 2;
+    const int blk = lane & 3;          // 16-row block of the step this lane loads
+    const int64_t cols = p.cols;
+
+    // this warp's tasks: first, first - wstride, ... >= t0
+    int64_t t0, first, wstride;
+    if (p.strided) {
+        t0 = 0;
+        wstride = (int64_t)p.num_ctas * kColWarps;
+        first = p.num_tasks - 1 - ((int64_t)blockIdx.x * kColWarps + warp);
+    } else {
+        t0 = (p.num_tasks * blockIdx.x) / p.num_ctas;
+        wstride = kColWarps;
+        first = (p.num_tasks * (blockIdx.x + 1)) / p.num_ctas - 1 - warp;
+    }
+    const int64_t ntask = first < t0 ? 0 : (first - t0) / wstride + 1;
+
+    // The current task is row task rt, column strip `strip`, of group g; the walk only
+    // goes backwards, wstride tasks at a time.
+    int g = 0, rt = 0, strip = 0;
+    auto locate = [&](ColTask& ct) {
+        if (MAXG > 1) {
+            while (g > 0 && rt < p.task_off[g]) --g;
+        }
+        ct.goff = p.row_off[g];
+        ct.grows = p.row_off[g + 1] - ct.goff;
+        ct.row0 = ct.goff + (rt - p.task_off[g]) * kTaskRows;
+        const int left = ct.goff + ct.grows - ct.row0;
+        ct.nrows = left >= kTaskRows ? kTaskRows : left;
+        ct.c0 = strip * kTaskCols;
+    };
+    auto step_back = [&]() {
+        strip -= p.back_strip;
+        rt -= p.back_rt;
+        if (strip < 0) { strip += p.strips; --rt; }
+    };
+
+    uint32_t va[16][2], vb[16][2];
+    // rows row0 + 16 * blk .. + 15 of columns c0 + 4 * quad .. + 3, zero where the
+    // block or the columns lie outside the task
+    const uint32_t row_bytes = (uint32_t)cols * 2u;
+    auto load = [&](const ColTask& ct, int step, uint32_t (&v)[16][2]) {
+        const int c = ct.c0 + 4 * quad;
+        const int r = kStepRows * step + 16 * blk;
+        const bool ok = r < ct.nrows && c < cols;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x + (int64_t)(ct.row0 + r) * cols + c);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (ok) {
+                const uint2 w = ldg64_stream(src);
+                v[i][0] = w.x;
+                v[i][1] = w.y;
+            } else {
+                v[i][0] = 0u;
+                v[i][1] = 0u;
+            }
+            src += row_bytes;
+        }
+    };
+    // amax of column 4q + j of a task for lane 4q + j (g is the task's group)
+    auto load_amax = [&](const ColTask& ct) -> float {
+        const int c = ct.c0 + 4 * quad + blk;
+        return c < cols ? p.amax_col[(int64_t)g * cols + c] : 0.0f;
+    };
+    // outer scales of the quad's four columns: each lane finds one, the quad shares them
+    auto outer_scales = [&](float a, float (&sc)[4]) {
+        const float mine = s_enc_of(a);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc[j] = __shfl_sync(0xFFFFFFFFu, mine, (lane & ~3) | j);
+    };
+
+    ColTask cur;
+    int step = 0;
+    if (ntask > 0) {
+        rt = (int)(first / p.strips);
+        strip = (int)(first - (int64_t)rt * p.strips);
+        if (MAXG > 1) g = group_of_task(p, rt);
+        locate(cur);
+        step = (cur.nrows - 1) / kStepRows;   // steps go backwards too
+        load(cur, step, va);   // x is read-only for the whole chain: load before the row pass ends
+    }
+
+    griddep_wait();
+    if (blockIdx.x == 0 && p.absmax) {
+        for (int i = tid; i < p.nbuf; i += kColThreads) {
+            const float d = __fmul_rn(p.absmax[i], p.decay);
+            const float o = p.obs[i];
+            p.absmax[i] = d > o ? d : o;
+        }
+    }
+    __syncthreads();   // rcp_tab
+    if (ntask == 0) return;
+
+    uint8_t* xc = col_stage + warp * kColStageBytes;
+    uint8_t* xs = xc + kTaskCols * 128;
+    // This lane's slots: column 4q+j, block kb = 4*step + blk goes to
+    // stage_off(4q+j, kb) = xq + 128j + 16*(hg ^ j), hg = (kb >> 1) ^ G(q), where
+    // g(4q+j) = j ^ G(q) with G(q) = 4(q & 1) ^ (q & 6); its scale byte to
+    // xsq + 16j + 4*step.
+    uint8_t* xq = xc + 512 * quad + 8 * (blk & 1);
+    uint8_t* xsq = xs + 64 * quad + blk;
+    const int gq = (4 * (quad & 1)) ^ (quad & 6);
+    const uint64_t pol_out = l2_evict_first();
+    float sc[4];
+    outer_scales(load_amax(cur), sc);
+
+    int64_t k = 0;   // tasks finished
+    // One step on the rows in `v` while the next step's rows load into `vn`; the
+    // loop alternates the two buffers. Returns false after the last step.
+    auto run_step = [&](uint32_t (&v)[16][2], uint32_t (&vn)[16][2]) -> bool {
+        // prefetch the next step: of this task, or the last step of the next task
+        ColTask nxt = cur;
+        int nstep = step - 1;
+        float a_nxt = 0.0f;
+        const bool more = step > 0 || k + 1 < ntask;
+        if (step == 0 && more) {
+            step_back();
+            locate(nxt);
+            nstep = (nxt.nrows - 1) / kStepRows;
+            a_nxt = load_amax(nxt);
+        }
+        if (more) load(nxt, nstep, vn);
+
+        // block amax of the four columns over this lane's 16 rows
+        uint32_t m[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint32_t t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = absmax2(v[i][w], v[i + 8][w]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) t[i] = absmax2(t[i], t[i + 4]);
+            t[0] = absmax2(t[0], t[2]);
+            t[1] = absmax2(t[1], t[3]);
+            m[w] = absmax2(t[0], t[1]) & 0x7FFF7FFFu;
+        }
+        uint32_t sf01, sf23;
+        float e[4];
+        block_pair_scales_x2(bf16_lo(m[0]), bf16_hi(m[0]), sc[0], sc[1], sf01, e[0], e[1], rcp_tab);
+        block_pair_scales_x2(bf16_lo(m[1]), bf16_hi(m[1]), sc[2], sc[3], sf23, e[2], e[3], rcp_tab);
+
+        // codes and scales of this lane's block of each column -> staging
+        const int hg = (2 * step + (blk >> 1)) ^ gq;
+        uint8_t* xsb = xsq + 4 * step;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int w = j >> 1;
+            const uint32_t lo = (j & 1) ? encode8_strided<true>(v, 0, w, e[j]) : encode8_strided<false>(v, 0, w, e[j]);
+            const uint32_t hi = (j & 1) ? encode8_strided<true>(v, 8, w, e[j]) : encode8_strided<false>(v, 8, w, e[j]);
+            *reinterpret_cast<uint2*>(xq + 128 * j + 16 * (hg ^ j)) = make_uint2(lo, hi);
+            xsb[16 * j] = (uint8_t)(((j < 2) ? sf01 : sf23) >> (8 * (j & 1)));
+        }
+
+        if (step == 0) {
+            // task done: write the task's columns out of staging
+            __syncwarp();
+            const int nblk = cur.nrows / 16;
+            const int lrow = cur.row0 - cur.goff;
+            const int64_t gq = cols * cur.goff / 2 + lrow / 2;    // column 0's code bytes, then
+            const int64_t cstride = cur.grows / 2;                //   one column every cstride
+            const bool wide = p.q_col_32 && (cur.grows & 63) == 0;
+            if (wide) {
+                // 32-byte aligned, nblk a multiple of 4: 8 lanes per column, 16 bytes
+                // each, so one store covers four columns' whole segments
+                const int k = lane & 7;
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int cl = 4 * it + (lane >> 3);
+                    const int c = cur.c0 + cl;
+                    if (c < cols && 2 * k < nblk) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(xc + stage_off(cl, 2 * k));
+                        stg16_ef(p.q_col + gq + (int64_t)c * cstride + 16 * k, a, pol_out);
+                    }
+                }
+            }
+            // lane j: column j's scales (and its codes when not aligned for the above)
+            const int c = cur.c0 + lane;
+            if (c < cols) {
+                uint8_t* q = p.q_col + gq + (int64_t)c * cstride;
+                uint8_t* sf = p.sf_col + cols * cur.goff / 16 + (int64_t)c * (cur.grows / 16) + lrow / 16;
+                if (!wide) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (i < nblk) {
+                            const uint2 a = *reinterpret_cast<const uint2*>(xc + stage_off(lane, i));
+                            stg8_ef(q + 8 * i, a.x, a.y, pol_out);
+                        }
+                    }
+                }
+                const uint4 s16 = *reinterpret_cast<const uint4*>(xs + 16 * lane);
+                if (nblk == 16 && (reinterpret_cast<uintptr_t>(sf) & 15u) == 0) {
+                    stg16_ef(sf, s16, pol_out);
+                } else {
+                    const uint32_t sw[4] = {s16.x, s16.y, s16.z, s16.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (4 * i < nblk) stg_bytes(sf + 4 * i, sw[i], min(4, nblk - 4 * i));
+                }
+            }
+            __syncwarp();
+            ++k;
+            if (more) {
+                cur = nxt;
+                outer_scales(a_nxt, sc);
+            }
+        }
+        step = nstep;
+        return more;
+    };
+    while (run_step(va, vb) && run_step(vb, va)) {
+    }
+}
+
+}  // namespace nvfp4pt

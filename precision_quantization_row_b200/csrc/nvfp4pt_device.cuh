@@ -318,12 +318,95 @@ __device__ __forceinline__ void block_pair_scales(float b0, float b1, float s0, 
     e1 = enc_of(sf01 >> 8, d1, s1, tab);
 }
 
+// ------------------------------------------------- packed two-lane binary32
+// One 64-bit register holds two binary32 lanes (lo, hi); the f32x2 instructions
+// round each lane exactly as the scalar instruction would.
+
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi)
+{
+    unsigned long long v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+
+__device__ __forceinline__ void unpack2(unsigned long long v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// a * b + c per lane, one rounding
+__device__ __forceinline__ unsigned long long fma_f32x2(unsigned long long a, unsigned long long b,
+                                                        unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// block_pair_scales with the two blocks in the lanes of packed instructions. Same
+// arithmetic step for step: RN(b/6) by div6's three operations (the remainder as
+// fma(q0, -6, b), equal to fma(-q0, 6, b)), times s, the E4M3 codes, and the quotient
+// s / d by div_by_e4m3's correction step written on the negated reciprocal -y:
+// q0n = s*(-y) = -RN(s*y), r = fma(q0n, d, s) = RN(s - q0*d), and
+// fma(r, -y, q0n) = -RN(q0 + r*y), negated back where it is clamped.
+__device__ __forceinline__ void block_pair_scales_x2(float b0, float b1, float s0, float s1, uint32_t& sf01,
+                                                     float& e0, float& e1, const uint32_t* tab)
+{
+    const unsigned long long r6 = pack2(0x1.555556p-3f, 0x1.555556p-3f);   // RN(1/6)
+    const unsigned long long b = pack2(b0, b1);
+    const unsigned long long q0 = mul_f32x2(b, r6);
+    const unsigned long long rem = fma_f32x2(q0, pack2(-6.0f, -6.0f), b);
+    const unsigned long long q1 = fma_f32x2(rem, r6, q0);
+    const unsigned long long s = pack2(s0, s1);
+    float u0, u1;
+    unpack2(mul_f32x2(q1, s), u0, u1);
+    sf01 = e4m3x2(u0, u1);
+    float d0, d1;
+    e4m3x2_decode(sf01, d0, d1);
+    const uint32_t db0 = __float_as_uint(d0), db1 = __float_as_uint(d1);
+    // -RN(1/d): the table entry with d's power of two taken out and the sign set
+    const float ny0 = __uint_as_float(tab[(db0 >> 20) & 7u] + 0xBF800000u - (db0 & 0x7F800000u));
+    const float ny1 = __uint_as_float(tab[(db1 >> 20) & 7u] + 0xBF800000u - (db1 & 0x7F800000u));
+    const unsigned long long ny = pack2(ny0, ny1);
+    const unsigned long long q0n = mul_f32x2(s, ny);
+    const unsigned long long r = fma_f32x2(q0n, pack2(d0, d1), s);
+    float qn0, qn1;
+    unpack2(fma_f32x2(r, ny, q0n), qn0, qn1);
+    e0 = (sf01 & 0xFFu) ? fminf(-qn0, FLT_MAX) : 0.0f;
+    e1 = (sf01 & 0xFF00u) ? fminf(-qn1, FLT_MAX) : 0.0f;
+}
+
+// Codes of four scaled pairs (y[2i], y[2i+1]) -> one word, y[j] in bits 4j..4j+3.
+__device__ __forceinline__ uint32_t e2m1x8_packed(const float (&y)[8])
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(r) : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    return r;
+}
+
 // Codes of the 8 elements held in 4 bf16 words with one multiplier: one word,
 // element i in bits 4i..4i+3.
 __device__ __forceinline__ uint32_t encode8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float e)
 {
-    return pack4(code_pair(bf16_lo(w0), bf16_hi(w0), e), code_pair(bf16_lo(w1), bf16_hi(w1), e),
-                 code_pair(bf16_lo(w2), bf16_hi(w2), e), code_pair(bf16_lo(w3), bf16_hi(w3), e));
+    float y[8];
+    mul2(y[0], y[1], bf16_lo(w0), bf16_hi(w0), e);
+    mul2(y[2], y[3], bf16_lo(w1), bf16_hi(w1), e);
+    mul2(y[4], y[5], bf16_lo(w2), bf16_hi(w2), e);
+    mul2(y[6], y[7], bf16_lo(w3), bf16_hi(w3), e);
+    return e2m1x8_packed(y);
 }
 
 // Codes of one column over 8 consecutive rows, the column being the low (hi=false) or
@@ -332,8 +415,12 @@ template <bool HI>
 __device__ __forceinline__ uint32_t encode8_col(const uint32_t* x, float e)
 {
     auto v = [&](int i) { return HI ? bf16_hi(x[i]) : bf16_lo(x[i]); };
-    return pack4(code_pair(v(0), v(1), e), code_pair(v(2), v(3), e), code_pair(v(4), v(5), e),
-                 code_pair(v(6), v(7), e));
+    float y[8];
+    mul2(y[0], y[1], v(0), v(1), e);
+    mul2(y[2], y[3], v(2), v(3), e);
+    mul2(y[4], y[5], v(4), v(5), e);
+    mul2(y[6], y[7], v(6), v(7), e);
+    return e2m1x8_packed(y);
 }
 
 // ---------------------------------------------------------------- memory ops
@@ -352,6 +439,28 @@ __device__ __forceinline__ void ldg256_stream(const void* p, uint32_t (&v)[8])
     asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
                  : "l"(p));
+}
+
+// Stores of outputs that nothing in the cast reads again, marked evict-first in L2 so
+// that they do not push out the lines of x that the column pass is about to read.
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void stg16_ef(uint8_t* p, uint4 v, uint64_t pol)   // 16-byte aligned
+{
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void stg8_ef(uint8_t* p, uint32_t a, uint32_t b, uint64_t pol)   // 8-byte aligned
+{
+    asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" :: "l"(p), "r"(a), "r"(b), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void stg1_ef(uint8_t* p, uint32_t v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.u8 [%0], %1, %2;" :: "l"(p), "r"(v), "l"(pol) : "memory");
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -383,6 +492,14 @@ __device__ __forceinline__ void stg16(uint8_t* p, uint32_t a, uint32_t b, uint32
         asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p), "r"(a), "r"(b) : "memory");
         asm volatile("st.global.v2.u32 [%0], {%1, %2};" :: "l"(p + 8), "r"(c), "r"(d) : "memory");
     }
+}
+
+// 32 bytes to a 32-byte aligned address in one store.
+__device__ __forceinline__ void stg32(uint8_t* p, uint4 a, uint4 b)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "l"(p), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
 }
 
 __device__ __forceinline__ void stg8(uint8_t* p, uint32_t a, uint32_t b)

@@ -399,29 +399,41 @@ __global__ void __launch_bounds__(kThreads, 2) pass2_encode(const __grid_constan
         }
         const int failed = __syncthreads_or(!ok);
         if (!failed && do_col) {
-            // coalesced write-back: 4 lanes per column (64 contiguous bytes), then 8 scale bytes
+            // write-back from the staging area: 64 contiguous code bytes and 8 scale bytes
+            // per column of the tile
             const int64_t lrow = cur.r0 - cur.goff;            // first row inside the group
             const int64_t qstride = cur.grows / 2, sstride = cur.grows / 16;
-            uint8_t* qbase = p.q_col + cols * (int64_t)cur.goff / 2 + lrow / 2;
-            uint8_t* sbase = p.sf_col + cols * (int64_t)cur.goff / 16 + lrow / 16;
-            const int qbytes = cur.nr / 2;                      // code bytes of this tile per column
+            uint8_t* qtile = p.q_col + cols * (int64_t)cur.goff / 2 + lrow / 2 + cur.c0 * qstride;
+            uint8_t* stile = p.sf_col + cols * (int64_t)cur.goff / 16 + lrow / 16 + cur.c0 * sstride;
+            const bool full = cur.nr == kTile && cur.nc == kTile;
+            if (full && ((reinterpret_cast<uintptr_t>(qtile) | (uintptr_t)qstride) & 31u) == 0) {
+                // one 32-byte half-column per thread
+                const int col = tid >> 1, h = tid & 1, sw = (col >> 1) & 3;
+                const uint8_t* src = ccode + col * 64;
+                const uint4 a = *reinterpret_cast<const uint4*>(src + 16 * ((2 * h) ^ sw));
+                const uint4 b = *reinterpret_cast<const uint4*>(src + 16 * ((2 * h + 1) ^ sw));
+                stg32(qtile + (int64_t)col * qstride + 32 * h, a, b);
+            } else {
+                const int qbytes = cur.nr / 2;                  // code bytes of this tile per column
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int i = tid + kThreads * j;
-                const int col = i >> 2, q = i & 3;
-                if (col < cur.nc && 16 * q < qbytes) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(ccode + col * 64 + 16 * (q ^ ((col >> 1) & 3)));
-                    uint8_t* dst = qbase + (cur.c0 + col) * qstride + 16 * q;
-                    if (16 * q + 16 <= qbytes) stg16(dst, v.x, v.y, v.z, v.w);
-                    else stg8(dst, v.x, v.y);
+                for (int j = 0; j < 2; ++j) {
+                    const int i = tid + kThreads * j;
+                    const int col = i >> 2, q = i & 3;
+                    if (col < cur.nc && 16 * q < qbytes) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(ccode + col * 64 + 16 * (q ^ ((col >> 1) & 3)));
+                        uint8_t* dst = qtile + (int64_t)col * qstride + 16 * q;
+                        if (16 * q + 16 <= qbytes) stg16(dst, v.x, v.y, v.z, v.w);
+                        else stg8(dst, v.x, v.y);
+                    }
                 }
             }
             if (tid < cur.nc) {
                 const uint2 v = *reinterpret_cast<const uint2*>(cscale + tid * 8);
-                uint8_t* dst = sbase + (cur.c0 + tid) * sstride;
+                uint8_t* dst = stile + (int64_t)tid * sstride;
                 const int nb = cur.nr / 16;
-                if (nb == 8 && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0) stg8(dst, v.x, v.y);
-                else {
+                if (nb == 8 && ((reinterpret_cast<uintptr_t>(stile) | (uintptr_t)sstride) & 7u) == 0) {
+                    stg8(dst, v.x, v.y);
+                } else {
                     stg_bytes(dst, v.x, nb < 4 ? nb : 4);
                     if (nb > 4) stg_bytes(dst + 4, v.y, nb - 4);
                 }

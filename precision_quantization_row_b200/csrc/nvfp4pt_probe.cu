@@ -93,6 +93,46 @@ __global__ void e4m3_div_kernel(int e_lo, int e_hi, unsigned long long* mismatch
     if (bad) atomicAdd(mismatches, bad);
 }
 
+// Both forms of the block-scale step on the same (b0, b1, s0, s1); counts the codes and
+// multipliers that differ. Thread (e, m) takes s0 = 2^e-binade significand m and s1 a
+// second significand of the same binade; b0 runs over all bf16 magnitudes, b1 the
+// other way round. The first thread also takes s = FLT_MAX and s = 1.
+__device__ unsigned long long pair_scales_diff(float s0, float s1, const uint32_t* tab)
+{
+    unsigned long long bad = 0;
+    for (uint32_t h = 0; h < 0x7F80u; ++h) {
+        const float b0 = __uint_as_float(h << 16);
+        const float b1 = __uint_as_float((0x7F7Fu - h) << 16);
+        uint32_t sfa, sfb;
+        float ea0, ea1, eb0, eb1;
+        block_pair_scales(b0, b1, s0, s1, sfa, ea0, ea1, tab);
+        block_pair_scales_x2(b0, b1, s0, s1, sfb, eb0, eb1, tab);
+        bad += ((sfa & 0xFFFFu) != (sfb & 0xFFFFu)) + (__float_as_uint(ea0) != __float_as_uint(eb0)) +
+               (__float_as_uint(ea1) != __float_as_uint(eb1));
+    }
+    return bad;
+}
+
+__global__ void pair_scales_kernel(int e_lo, int e_hi, uint32_t stride, unsigned long long* mismatches)
+{
+    __shared__ uint32_t tab[8];
+    init_rcp_table(tab);
+    __syncthreads();
+    const uint64_t per = ((1u << 23) - 1) / stride + 1;   // significands 0, stride, ... < 2^23
+    const uint64_t total = (uint64_t)(e_hi - e_lo + 1) * per;
+    unsigned long long bad = 0;
+    const uint64_t t0 = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (uint64_t i = t0; i < total; i += (uint64_t)gridDim.x * blockDim.x) {
+        const uint32_t e = (uint32_t)(e_lo + i / per);
+        const uint32_t m = (uint32_t)(i % per) * stride;
+        const float s0 = __uint_as_float((e << 23) | m);
+        const float s1 = __uint_as_float((e << 23) | ((m * 2654435761u) & 0x7FFFFFu));
+        bad += pair_scales_diff(s0, s1, tab);
+    }
+    if (t0 == 0) bad += pair_scales_diff(FLT_MAX, 1.0f, tab) + pair_scales_diff(1.0f, FLT_MAX, tab);
+    if (bad) atomicAdd(mismatches, bad);
+}
+
 nvfp4pt_status arch_ok()
 {
     int dev = 0, major = 0, minor = 0;
@@ -152,6 +192,18 @@ nvfp4pt_status nvfp4pt_probe_e4m3_div(int exp_lo, int exp_hi, unsigned long long
     if (st != NVFP4PT_OK) return st;
     if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), stream) != cudaSuccess) return NVFP4PT_ERR_CUDA;
     e4m3_div_kernel<<<148 * 8, 256, 0, stream>>>(exp_lo, exp_hi, mismatches);
+    return last();
+}
+
+nvfp4pt_status nvfp4pt_probe_pair_scales(int exp_lo, int exp_hi, unsigned int stride, unsigned long long* mismatches,
+                                         cudaStream_t stream)
+{
+    if (!mismatches) return NVFP4PT_ERR_NULL;
+    if (exp_lo < 1 || exp_hi > 254 || exp_lo > exp_hi || stride < 1) return NVFP4PT_ERR_SHAPE;
+    nvfp4pt_status st = arch_ok();
+    if (st != NVFP4PT_OK) return st;
+    if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), stream) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    pair_scales_kernel<<<148 * 4, 256, 0, stream>>>(exp_lo, exp_hi, (uint32_t)stride, mismatches);
     return last();
 }
 

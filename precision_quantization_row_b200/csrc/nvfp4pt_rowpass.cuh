@@ -1,6 +1,6 @@
 // Row pass of the NVFP4 per-token cast (sm_100a): one read of x gives the per-row
 // amax, the complete rowwise encode (codes + E4M3 scales) and the per-column amax
-// (per token group). The columnwise encode follows in pass2_encode.
+// (per token group). The columnwise encode follows in the column pass (colpass).
 //
 // Why here: a row's outer amax needs only that row, so a CTA that holds whole rows
 // can encode them as soon as its own reduction ends, from registers. That moves
@@ -9,10 +9,16 @@
 //
 // Layout of the work: a "sweep" is `rps` whole rows covered once by the CTA's 512
 // threads (tpr threads per row, a multiple of 32, each holding BT 16-element blocks
-// of its row); a "batch" is S sweeps. A CTA owns a contiguous run of batches, and
-// prefetches the next batch (one 256-bit load per block) while it reduces and encodes
-// the current one. A batch has S * rps rows, a divisor of 16, so it never straddles a
-// token group (group offsets are multiples of 16).
+// of its row); a "batch" is S sweeps. A CTA prefetches the next batch (one 256-bit
+// load per block) while it reduces and encodes the current one. A batch has S * rps
+// rows, a divisor of 16, so it never straddles a token group (group offsets are
+// multiples of 16).
+//
+// Order of the batches: with one token group the CTAs take batches c, c + num_ctas,
+// ... so that the grid sweeps x from top to bottom as one front, and the bottom of x
+// is what L2 holds when the column pass starts there. With several groups a CTA owns
+// a contiguous run of batches instead, so that its column partials change group (and
+// go out to amax_col) about once per group rather than once per batch.
 #pragma once
 
 #include "nvfp4pt_device.cuh"
@@ -32,6 +38,7 @@ struct RowParams {
     int32_t num_ctas;
     int32_t num_groups;
     int32_t do_row;      // write rowwise codes and scales
+    int32_t strided;     // batches c, c + num_ctas, ... (else a contiguous run per CTA)
     const uint16_t* x;
     float* amax_row;     // [rows], written directly (not accumulated)
     uint8_t* q_row;
@@ -87,9 +94,17 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
     const int64_t cols = p.cols;
 
     const int64_t nb = p.num_batches;
-    const int64_t b0 = (nb * blockIdx.x) / p.num_ctas;
-    const int64_t b1 = (nb * (blockIdx.x + 1)) / p.num_ctas;
-    if (b0 >= b1) return;
+    int64_t b0, bstep, nbat;   // this CTA's batches: b0 + k * bstep, k < nbat
+    if (p.strided) {
+        b0 = blockIdx.x;
+        bstep = p.num_ctas;
+        nbat = b0 < nb ? (nb - 1 - b0) / bstep + 1 : 0;
+    } else {
+        b0 = (nb * blockIdx.x) / p.num_ctas;
+        bstep = 1;
+        nbat = (nb * (blockIdx.x + 1)) / p.num_ctas - b0;
+    }
+    if (nbat <= 0) return;
 
     bool valid[BT];
     int bj[BT];
@@ -101,6 +116,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
 
     uint32_t va[S][BT][8];
     uint32_t vb[S][BT][8];
+    const uint64_t pol_out = l2_evict_first();   // row outputs: not read again
     auto load = [&](int64_t batch, uint32_t (&v)[S][BT][8]) {
         const int64_t r0 = batch * rows_per_batch;
 #pragma unroll
@@ -147,8 +163,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
     };
 
     int g_cur = group_of_row(p, b0 * rows_per_batch);
-    auto process = [&](int64_t batch, uint32_t (&cur)[S][BT][8], uint32_t (&nxt)[S][BT][8]) {
-        if (batch + 1 < b1) load(batch + 1, nxt);
+    auto process = [&](int64_t batch, bool more, uint32_t (&cur)[S][BT][8], uint32_t (&nxt)[S][BT][8]) {
+        if (more) load(batch + bstep, nxt);
         const int64_t r0 = batch * rows_per_batch;
 
         // block amaxes (kept for the encode), row partials (one per warp and row),
@@ -200,19 +216,19 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
                                   sv[sa], sv[sb], qa0, qa1, qb0, qb1, sf, rcp_tab);
                 if (valid[ba]) {
                     const int64_t row = r0 + sa * p.rps + rsw;
-                    stg8(p.q_row + row * (cols / 2) + 8 * (int64_t)bj[ba], qa0, qa1);
-                    p.sf_row[row * (cols / 16) + bj[ba]] = (uint8_t)sf;
+                    stg8_ef(p.q_row + row * (cols / 2) + 8 * (int64_t)bj[ba], qa0, qa1, pol_out);
+                    stg1_ef(p.sf_row + row * (cols / 16) + bj[ba], sf & 0xFFu, pol_out);
                 }
                 if (i + 1 < S * BT && valid[bb]) {
                     const int64_t row = r0 + sb * p.rps + rsw;
-                    stg8(p.q_row + row * (cols / 2) + 8 * (int64_t)bj[bb], qb0, qb1);
-                    p.sf_row[row * (cols / 16) + bj[bb]] = (uint8_t)(sf >> 8);
+                    stg8_ef(p.q_row + row * (cols / 2) + 8 * (int64_t)bj[bb], qb0, qb1, pol_out);
+                    stg1_ef(p.sf_row + row * (cols / 16) + bj[bb], (sf >> 8) & 0xFFu, pol_out);
                 }
             }
         }
 
         // the column partials belong to the batch's token group
-        const int g_next = (batch + 1 < b1) ? group_of_row(p, (batch + 1) * rows_per_batch) : -1;
+        const int g_next = more ? group_of_row(p, (batch + bstep) * rows_per_batch) : -1;
         if (g_next != g_cur) {
             flush(g_cur);
             g_cur = g_next;
@@ -221,14 +237,14 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
 
     // the next batch loads into vb while va is reduced and encoded, then moves over
     load(b0, va);
-    for (int64_t batch = b0; batch < b1; ++batch) {
-        process(batch, va, vb);
+    for (int64_t k = 0; k < nbat; ++k) {
+        process(b0 + k * bstep, k + 1 < nbat, va, vb);
 #pragma unroll
         for (int s = 0; s < S; ++s)
 #pragma unroll
             for (int b = 0; b < BT; ++b)
 #pragma unroll
-                for (int k = 0; k < 8; ++k) va[s][b][k] = vb[s][b][k];
+                for (int i = 0; i < 8; ++i) va[s][b][i] = vb[s][b][i];
     }
 }
 

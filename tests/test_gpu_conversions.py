@@ -125,3 +125,15 @@ def test_block_scale_division_matches_ieee(lo, hi):
                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     assert int(bad.item()) == 0
+
+
+def test_packed_block_scales_match_scalar():
+    """The block-scale step in the packed two-lane form the column pass uses equals the
+    scalar form (pinned to the oracle by the parity tests) bit for bit: every bf16
+    block amax, against every 4093rd significand of s in every binade that s_enc can
+    take (2688 / max bf16 ~ 2^-117 up to FLT_MAX), plus s = FLT_MAX and s = 1."""
+    bad = torch.zeros(1, dtype=torch.int64, device="cuda")
+    st = nv.lib().nvfp4pt_probe_pair_scales(10, 254, 4093, ctypes.c_void_p(bad.data_ptr()),
+                                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    assert int(bad.item()) == 0
