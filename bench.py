@@ -44,7 +44,22 @@ def workload_name(m: int, k: int) -> str:
     return f"llm_activation_{m}x{k}_bf16_rowcol_decay0.99"
 PROFILE_JSON = os.path.join(ROOT, "profiles", "nvfp4pt_cast_llm_16384x8192.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "precision_quantization_row_b200", "csrc", f)
-                  for f in ("nvfp4pt_api.cu", "nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh")]
+                  for f in ("nvfp4pt_api.cu", "nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh", "nvfp4pt_rowpass.cuh",
+                            "nvfp4pt_colpass.cuh")]
+# The cast's launches on rows of up to 16384 elements, in order (nvfp4pt_timing.h):
+# zeroing, the row pass, the column pass.
+KERNELS = ("pass0_zero", "rowpass", "colpass")
+
+
+def kernel_bytes(name: str, m: int, k: int) -> int:
+    """Algorithmic bytes of one launch: what the kernel must read and write at least.
+    Row pass: x once; row codes, row scales, row amax; the column amax vector.
+    Column pass: x once and the column amax; column codes and scales."""
+    if name == "rowpass":
+        return 2 * m * k + m * k // 2 + m * k // 16 + 4 * m + 4 * k
+    if name == "colpass":
+        return 2 * m * k + 4 * k + m * k // 2 + m * k // 16
+    return 4 * k
 
 
 def kernel_source_sha() -> str:
@@ -63,14 +78,14 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def ncu_traffic():
-    """DRAM bytes per cast from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+def ncu_traffic(kernel: str):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary,
+    if it was taken on the current kernel sources (else None)."""
     try:
         with open(PROFILE_JSON) as f:
             d = json.load(f)
         if d.get("kernel_source_sha") == kernel_source_sha():
-            return d.get("dram_bytes_per_cast")
+            return d["kernels"][kernel]["dram_bytes_per_launch"]
     except Exception:
         pass
     return None
@@ -227,7 +242,26 @@ def run_gpu(args, dist: Dist) -> dict | None:
 
     with ClockSampler(dev.index) as clk:
         secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
-    launches = 3 * args.steps  # zero, amax pass, encode pass per cast
+    launches = nv.CAST_LAUNCHES * args.steps  # zero, row pass, column pass per cast
+
+    # Per-kernel times: the same casts through the timed entry, which records an event
+    # before the first launch and after each launch on the casts' stream.
+    kt_steps = min(args.steps, 200)
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nv.CAST_LAUNCHES + 1)] for _ in range(kt_steps)]
+    for row in kevs:
+        for e in row:
+            e.record(stream)
+
+    def run_kernels():
+        for i in range(kt_steps):
+            nv.quantize_timed(xs[i & 1], kevs[i], absmax=buf, decay=DECAY, out=outs[i & 1], workspace=ws,
+                              stream=stream)
+        kevs[-1][-1].synchronize()
+        return 0.0
+
+    timed_region(dist, run_kernels, lambda: torch.cuda.synchronize(dev))
+    kernel_ms = {name: dist.max(sum(row[j].elapsed_time(row[j + 1]) for row in kevs) / kt_steps)
+                 for j, name in enumerate(KERNELS)}
 
     # end to end through the public call with host buffers: pinned H2D of the input,
     # the cast, D2H of every output (codes, scales, amax vectors, buffer)
@@ -268,7 +302,10 @@ def run_gpu(args, dist: Dist) -> dict | None:
         return None
     peak, peak_kind = measured_peak()
     per_cast = secs / args.steps
-    achieved = algo_bytes(M, K) / per_cast / 1e9
+    cast_achieved = algo_bytes(M, K) / per_cast / 1e9
+    dominant = max(("rowpass", "colpass"), key=lambda n: kernel_ms[n])
+    achieved = kernel_bytes(dominant, M, K) / (kernel_ms[dominant] / 1e3) / 1e9
+    traffic = ncu_traffic(dominant)
     elems = float(M) * K
     line = {
         "metric": "NVFP4 per-token cast: elems/s, achieved HBM GB/s, % of B200 HBM peak",
@@ -287,10 +324,16 @@ def run_gpu(args, dist: Dist) -> dict | None:
                    "absmax_decay": DECAY, "parallelism": f"replicas x{dist.world}",
                    "l2": f"inputs larger than L2 ({M * K * 2 / 1e6:.0f} MB each), 2 rotating input copies "
                          "and output sets"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": ncu_traffic(), "peak_source": peak_kind,
-                     "nominal_frac_8TBs": achieved / 8000.0,
-                     "algorithmic_bytes_per_cast": algo_bytes(M, K)},
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": kernel_bytes(dominant, M, K),
+                     "launch_us": kernel_ms[dominant] * 1e3,
+                     "kernels_us": {n: round(v * 1e3, 2) for n, v in kernel_ms.items()},
+                     "kernels_note": f"CUDA events around each launch, {kt_steps} casts; the launches "
+                                     "then run one after another",
+                     "cast": {"achieved": cast_achieved, "frac": cast_achieved / peak,
+                              "nominal_frac_8TBs": cast_achieved / 8000.0,
+                              "algorithmic_bytes_per_cast": algo_bytes(M, K)}},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),

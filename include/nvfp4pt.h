@@ -81,9 +81,11 @@ enum { NVFP4PT_ROWWISE = 1, NVFP4PT_COLWISE = 2 };
 NVFP4PT_API const char* nvfp4pt_status_string(nvfp4pt_status status);
 
 /* Bytes of device workspace a call with these sizes needs (num_groups = 1 for the
- * ungrouped and weight calls). The workspace holds per-call scratch (the observed
- * maxima of the absmax update and a device error word); it needs no initialisation
- * and its contents after a call are unspecified except for the error word. */
+ * ungrouped and weight calls): about num_groups * cols * 2 bytes plus a few hundred.
+ * The workspace holds per-call scratch (a device error word, the observed maxima of
+ * the absmax update, and the column maxima as bf16 while the columnwise cast runs);
+ * it needs no initialisation and its contents after a call are unspecified except for
+ * the error word. */
 NVFP4PT_API size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
 
 /*

@@ -35,6 +35,7 @@ EXPORTS = (
     "nvfp4pt_quantize_weight_2d", "nvfp4pt_update_absmax", "nvfp4pt_workspace_error",
     "nvfp4pt_probe_transitions", "nvfp4pt_probe_pairs", "nvfp4pt_probe_e4m3_decode", "nvfp4pt_probe_div6",
     "nvfp4pt_probe_e4m3_div", "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_probe_pair_scales",
+    "nvfp4pt_quantize_timed",
 )
 
 
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_probe_e4m3_div.argtypes = [I, I, P, P]
         L.nvfp4pt_quantize_grouped_noalloc.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, F, P]
         L.nvfp4pt_probe_pair_scales.argtypes = [I, I, ctypes.c_uint32, P, P]
+        L.nvfp4pt_quantize_timed.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, F, P, P, P]
         for name in EXPORTS[2:]:
             getattr(L, name).restype = I
         _lib = L
@@ -136,6 +138,30 @@ def quantize(x: torch.Tensor, flags: int = ROWWISE | COLWISE, absmax: torch.Tens
         _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("amax_col")), _ptr(absmax),
         ctypes.c_float(decay), _ptr(ws), _stream(stream, x.device))
     _check("nvfp4pt_quantize", st)
+    return out
+
+
+CAST_LAUNCHES = 3   # kernel launches of one quantize call (nvfp4pt_timing.h)
+
+
+def quantize_timed(x: torch.Tensor, events, flags: int = ROWWISE | COLWISE, absmax: torch.Tensor | None = None,
+                   decay: float = 0.0, out: dict | None = None, workspace: torch.Tensor | None = None,
+                   stream: torch.cuda.Stream | None = None) -> dict:
+    """nvfp4pt_quantize_timed: quantize with events[0] recorded before the first kernel
+    launch and events[i] after the i-th (CAST_LAUNCHES + 1 torch.cuda.Event objects,
+    created with enable_timing=True and already recorded once, so that they exist)."""
+    _require_cuda_bf16(x, "x")
+    if len(events) != CAST_LAUNCHES + 1:
+        raise ValueError(f"need {CAST_LAUNCHES + 1} events")
+    rows, cols = x.shape
+    out = _outputs(rows, cols, flags, x.device) if out is None else out
+    ws = new_workspace(rows, cols, 1, x.device) if workspace is None else workspace
+    evs = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    st = lib().nvfp4pt_quantize_timed(
+        _ptr(x), rows, cols, flags, _ptr(out.get("q_row")), _ptr(out.get("sf_row")), _ptr(out.get("amax_row")),
+        _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("amax_col")), _ptr(absmax),
+        ctypes.c_float(decay), _ptr(ws), _stream(stream, x.device), evs)
+    _check("nvfp4pt_quantize_timed", st)
     return out
 
 

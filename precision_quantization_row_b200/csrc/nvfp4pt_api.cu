@@ -8,6 +8,8 @@
 #include <mutex>
 
 #include "nvfp4pt.h"
+#include "nvfp4pt_timing.h"
+#include "nvfp4pt_internal.h"
 #include "nvfp4pt_kernels.cuh"
 #include "nvfp4pt_rowpass.cuh"
 #include "nvfp4pt_colpass.cuh"
@@ -97,9 +99,17 @@ nvfp4pt_status encode_map(CUtensorMap* map, const void* x, int64_t rows, int64_t
 }
 
 // Workspace layout: [0, 4) error word; [16, ...) observed maxima, one per buffer.
+// Workspace layout: the error word at 0, the observed maxima (one float per group) at
+// 16, then -- in a full workspace -- the row pass's bf16 column maxima [G, cols].
+int64_t pad4(int64_t n) { return (n + 3) & ~int64_t(3); }
+int64_t align256(int64_t n) { return (n + 255) & ~int64_t(255); }
+int64_t ws_small_bytes(int64_t groups) { return align256(16 + 4 * pad4(groups)); }
 uint32_t* ws_err(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 float* ws_obs(void* ws) { return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 16); }
-int64_t pad4(int64_t n) { return (n + 3) & ~int64_t(3); }
+uint16_t* ws_colmax(void* ws, int64_t groups)
+{
+    return reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + ws_small_bytes(groups));
+}
 
 template <typename Kernel, typename Params>
 cudaError_t launch(Kernel kernel, int grid, int smem, cudaStream_t stream, const Params& p, bool pdl,
@@ -182,8 +192,13 @@ cudaError_t launch_rowpass(const RowShape& rs, const RowParams<MAXG>& rp, cudaSt
 template <int MAXG>
 nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t* off, int G, int flags,
                         uint8_t* q_row, uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col,
-                        float* amax_col, float* absmax, float decay, bool w2d, void* ws, cudaStream_t stream)
+                        float* amax_col, float* absmax, float decay, bool w2d, void* ws, cudaStream_t stream,
+                        void* const* events = nullptr, bool full_ws = true)
 {
+    // events[0] before the first launch, events[i] after the i-th (measurement hook)
+    auto mark = [&](int i) -> bool {
+        return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
+    };
     DeviceState* dev = nullptr;
     nvfp4pt_status st = device_state(&dev);
     if (st != NVFP4PT_OK) return st;
@@ -192,14 +207,17 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
     const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
     // The 1D cast of rows up to kRowPassMaxCols wide encodes rows in the amax pass.
     const bool row_pass = !w2d && cols <= kRowPassMaxCols;
+    // bf16 column maxima in the workspace (8 columns per atomic), else fp32 atomics
+    uint16_t* colmax = (row_pass && do_col && full_ws) ? ws_colmax(ws, G) : nullptr;
 
     ZeroParams z;
     std::memset(&z, 0, sizeof z);
     if (do_row && !row_pass) { z.ptr[0] = reinterpret_cast<float4*>(amax_row); z.n4[0] = rows / 4; }
     if (do_col) { z.ptr[1] = reinterpret_cast<float4*>(amax_col); z.n4[1] = (int64_t)G * cols / 4; }
     if (absmax) { z.ptr[2] = reinterpret_cast<float4*>(ws_obs(ws)); z.n4[2] = pad4(G) / 4; }
+    if (colmax) { z.ptr[3] = reinterpret_cast<float4*>(colmax); z.n4[3] = (int64_t)G * cols * 2 / 16; }
     z.err = ws_err(ws);
-    if (launch_zero(stream, z) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    if (!mark(0) || launch_zero(stream, z) != cudaSuccess || !mark(1)) return NVFP4PT_ERR_CUDA;
 
     cudaError_t e;
     if (row_pass) {
@@ -220,10 +238,11 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         rp.amax_row = do_row ? amax_row : nullptr;
         rp.q_row = q_row;
         rp.sf_row = sf_row;
-        rp.amax_col = do_col ? amax_col : nullptr;
+        rp.amax_col = (do_col && !colmax) ? amax_col : nullptr;
+        rp.colmax = reinterpret_cast<uint32_t*>(colmax);
         rp.obs = absmax ? ws_obs(ws) : nullptr;
         for (int g = 0; g <= G; ++g) rp.row_off[g] = (int32_t)off[g];
-        if ((e = launch_rowpass<MAXG>(rs, rp, stream)) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+        if ((e = launch_rowpass<MAXG>(rs, rp, stream)) != cudaSuccess || !mark(2)) return NVFP4PT_ERR_CUDA;
 
         // Column pass: 256-row tasks per group (the last one ragged) x 32-column strips.
         // With nothing to encode it runs the running-buffer update alone (one CTA).
@@ -252,12 +271,13 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         cp.back_strip = (int32_t)(wstride % cp.strips);
         cp.x = static_cast<const uint16_t*>(x);
         cp.amax_col = amax_col;
+        cp.colmax = colmax;
         cp.q_col = q_col;
         cp.sf_col = sf_col;
         cp.absmax = absmax;
         cp.obs = ws_obs(ws);
         e = launch(colpass<MAXG>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
-        return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+        return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
     }
 
     P2Params<MAXG> p2;
@@ -286,10 +306,10 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
     p1.obs = absmax ? ws_obs(ws) : nullptr;
     if (do_col) e = launch(pass1_amax<MAXG, true>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
     else e = launch(pass1_amax<MAXG, false>, p1.geo.num_ctas, 0, stream, p1, true, kThreads);
-    if (e != cudaSuccess) return NVFP4PT_ERR_CUDA;
+    if (e != cudaSuccess || !mark(2)) return NVFP4PT_ERR_CUDA;
     if (w2d) e = launch(pass2_encode<MAXG, true>, p2.geo.num_ctas, kSmemPass2, stream, p2, true, kThreads);
     else e = launch(pass2_encode<MAXG, false>, p2.geo.num_ctas, kSmemPass2, stream, p2, true, kThreads);
-    return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+    return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 
 }  // namespace
@@ -315,15 +335,23 @@ const char* nvfp4pt_status_string(nvfp4pt_status s)
 size_t nvfp4pt_workspace_bytes(int64_t rows, int64_t cols, int num_groups)
 {
     (void)rows;
-    (void)cols;
     const int64_t g = num_groups < 1 ? 1 : num_groups;
-    const int64_t bytes = 16 + 4 * pad4(g);
-    return (size_t)((bytes + 255) & ~int64_t(255));
+    const int64_t c = cols < 0 ? 0 : cols;
+    return (size_t)(ws_small_bytes(g) + align256(g * c * 2));
 }
 
 nvfp4pt_status nvfp4pt_quantize(const void* x, int64_t rows, int64_t cols, int flags, uint8_t* q_row,
                                 uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col, float* amax_col,
                                 float* absmax_buf, float decay, void* workspace, cudaStream_t stream)
+{
+    return nvfp4pt_quantize_timed(x, rows, cols, flags, q_row, sf_row, amax_row, q_col, sf_col, amax_col, absmax_buf,
+                                  decay, workspace, stream, nullptr);
+}
+
+nvfp4pt_status nvfp4pt_quantize_timed(const void* x, int64_t rows, int64_t cols, int flags, uint8_t* q_row,
+                                      uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col,
+                                      float* amax_col, float* absmax_buf, float decay, void* workspace,
+                                      cudaStream_t stream, void* const* events)
 {
     const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
     const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
@@ -339,13 +367,28 @@ nvfp4pt_status nvfp4pt_quantize(const void* x, int64_t rows, int64_t cols, int f
         return NVFP4PT_ERR_ALIGN;
     const int64_t off[2] = {0, rows};
     return run_cast<1>(x, rows, cols, off, 1, flags, q_row, sf_row, amax_row, q_col, sf_col, amax_col, absmax_buf,
-                       decay, false, workspace, stream);
+                       decay, false, workspace, stream, events);
 }
 
 nvfp4pt_status nvfp4pt_quantize_grouped(const void* x, int64_t rows, int64_t cols, const int64_t* offsets,
                                         int num_groups, int flags, uint8_t* q_row, uint8_t* sf_row,
                                         float* amax_row, uint8_t* q_col, uint8_t* sf_col, float* amax_col,
                                         float* absmax_bufs, float decay, void* workspace, cudaStream_t stream)
+{
+    return nvfp4pt::quantize_grouped_ws(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row, q_col,
+                                        sf_col, amax_col, absmax_bufs, decay, workspace, stream, true);
+}
+
+}  // extern "C"
+
+namespace nvfp4pt {
+
+size_t small_workspace_bytes(int num_groups) { return (size_t)ws_small_bytes(num_groups < 1 ? 1 : num_groups); }
+
+nvfp4pt_status quantize_grouped_ws(const void* x, int64_t rows, int64_t cols, const int64_t* offsets,
+                                   int num_groups, int flags, uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                   uint8_t* q_col, uint8_t* sf_col, float* amax_col, float* absmax_bufs, float decay,
+                                   void* workspace, cudaStream_t stream, bool full_ws)
 {
     const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
     const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
@@ -364,8 +407,12 @@ nvfp4pt_status nvfp4pt_quantize_grouped(const void* x, int64_t rows, int64_t col
     for (int g = 0; g < num_groups; ++g)
         if (offsets[g + 1] < offsets[g] || offsets[g] % 16) return NVFP4PT_ERR_GROUPS;
     return run_cast<kMaxGroups>(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row, q_col, sf_col,
-                                amax_col, absmax_bufs, decay, false, workspace, stream);
+                                amax_col, absmax_bufs, decay, false, workspace, stream, nullptr, full_ws);
 }
+
+}  // namespace nvfp4pt
+
+extern "C" {
 
 nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w, int64_t rows, int64_t cols, uint8_t* q_row,
                                           uint8_t* sf_row, float* amax_row, void* workspace, cudaStream_t stream)

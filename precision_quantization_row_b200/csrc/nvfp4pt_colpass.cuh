@@ -47,7 +47,9 @@ struct ColParams {
     int32_t back_rt;     // a warp's next task is wstride tasks back:
     int32_t back_strip;  //   wstride = back_rt * strips + back_strip, back_strip < strips
     const uint16_t* x;
-    const float* amax_col;   // [G, cols], final when the row pass has ended
+    float* amax_col;         // [G, cols] fp32: final when the row pass has ended, or (when colmax is
+                             //   set) written here from colmax
+    const uint16_t* colmax;  // [G, cols] bf16 column maxima left by the row pass, or null
     uint8_t* q_col;
     uint8_t* sf_col;
     float* absmax;           // [nbuf] running amax buffers, or null
@@ -181,7 +183,15 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
     // amax of column 4q + j of a task for lane 4q + j (g is the task's group)
     auto load_amax = [&](const ColTask& ct) -> float {
         const int c = ct.c0 + 4 * quad + blk;
-        return c < cols ? p.amax_col[(int64_t)g * cols + c] : 0.0f;
+        if (c >= cols) return 0.0f;
+        const int64_t i = (int64_t)g * cols + c;
+        return p.colmax ? __uint_as_float((uint32_t)p.colmax[i] << 16) : p.amax_col[i];
+    };
+    // With colmax, the fp32 amax_col output of (group, strip) comes from the warp that
+    // takes the group's first row task there: lane l holds column c0 + l's amax.
+    auto publish_amax = [&](const ColTask& ct, float a) {
+        const int c = ct.c0 + lane;
+        if (p.colmax && ct.row0 == ct.goff && c < cols) p.amax_col[(int64_t)g * cols + c] = a;
     };
     // outer scales of the quad's four columns: each lane finds one, the quad shares them
     auto outer_scales = [&](float a, float (&sc)[4]) {
@@ -223,7 +233,11 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
     const int gq = (4 * (quad & 1)) ^ (quad & 6);
     const uint64_t pol_out = l2_evict_first();
     float sc[4];
-    outer_scales(load_amax(cur), sc);
+    {
+        const float a = load_amax(cur);
+        publish_amax(cur, a);
+        outer_scales(a, sc);
+    }
 
     int64_t k = 0;   // tasks finished
     // One step on the rows in `v` while the next step's rows load into `vn`; the
@@ -322,6 +336,7 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
             ++k;
             if (more) {
                 cur = nxt;
+                publish_amax(cur, a_nxt);
                 outer_scales(a_nxt, sc);
             }
         }

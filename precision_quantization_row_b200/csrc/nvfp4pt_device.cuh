@@ -526,6 +526,14 @@ __device__ __forceinline__ void red_max_f32(float* p, uint32_t bits)
     atomicMax(reinterpret_cast<unsigned int*>(p), bits);
 }
 
+// Lane-wise atomic max of 8 non-negative bf16 values (four bf16x2 words) into 16-byte
+// aligned global memory: one reduction operation instead of eight.
+__device__ __forceinline__ void red_max_bf16x8(uint32_t* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("red.global.max.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};"
+                 :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 // ------------------------------------------------------------ mbarrier + TMA
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)

@@ -6,10 +6,12 @@
 //
 // The cast's scratch (an error word and one observed maximum per token group) lives
 // in g_scratch below instead of a caller-provided workspace; the kernels and the
-// launch sequence are exactly those of nvfp4pt_quantize_grouped.
+// launch sequence are those of nvfp4pt_quantize_grouped, with the column maxima
+// accumulated in amax_col itself (fp32 atomic max) for want of workspace room.
 #include <mutex>
 
 #include "nvfp4pt.h"
+#include "nvfp4pt_internal.h"
 
 namespace {
 
@@ -45,12 +47,15 @@ extern "C" nvfp4pt_status nvfp4pt_quantize_grouped_noalloc(
     float* absmax_bufs, float decay, cudaStream_t stream)
 {
     if (num_groups < 1 || num_groups > NVFP4PT_NOALLOC_MAX_GROUPS ||
-        nvfp4pt_workspace_bytes(rows, cols, num_groups) > NVFP4PT_NOALLOC_SCRATCH_BYTES)
+        nvfp4pt::small_workspace_bytes(num_groups) > NVFP4PT_NOALLOC_SCRATCH_BYTES)
         return NVFP4PT_ERR_GROUPS;
     void* scratch = nullptr;
     const nvfp4pt_status st = scratch_address(&scratch);
     if (st != NVFP4PT_OK) return st;
-    // The cast clears the scratch it accumulates into at the start of every call.
-    return nvfp4pt_quantize_grouped(x_bf16, rows, cols, offsets_host, num_groups, flags, q_row, sf_row, amax_row,
-                                    q_col, sf_col, amax_col, absmax_bufs, decay, scratch, stream);
+    // The cast clears the scratch it accumulates into at the start of every call. The
+    // scratch has no room for the bf16 column maxima of a full workspace, so the column
+    // maxima accumulate in amax_col by fp32 atomic max instead.
+    return nvfp4pt::quantize_grouped_ws(x_bf16, rows, cols, offsets_host, num_groups, flags, q_row, sf_row,
+                                        amax_row, q_col, sf_col, amax_col, absmax_bufs, decay, scratch, stream,
+                                        false);
 }

@@ -43,7 +43,8 @@ struct RowParams {
     float* amax_row;     // [rows], written directly (not accumulated)
     uint8_t* q_row;
     uint8_t* sf_row;
-    float* amax_col;     // [G, cols] accumulated with atomic max, or null
+    float* amax_col;     // [G, cols] accumulated with atomic max, or null (used when colmax is null)
+    uint32_t* colmax;    // [G, cols] bf16 column maxima accumulated with 8-wide atomic max, or null
     float* obs;          // [G] accumulated with atomic max, or null
     int32_t row_off[MAXG + 1];
 };
@@ -144,7 +145,21 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
 
     auto flush = [&](int g) {
         if (!waited) { griddep_wait(); waited = true; }
-        if (p.amax_col) {
+        if (p.colmax) {
+#pragma unroll
+            for (int b = 0; b < BT; ++b) {
+                if (!valid[b]) continue;
+                uint32_t* dst = p.colmax + ((int64_t)g * cols + 16 * (int64_t)bj[b]) / 2;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t w0 = colacc[b][4 * h] & 0x7FFF7FFFu, w1 = colacc[b][4 * h + 1] & 0x7FFF7FFFu;
+                    const uint32_t w2 = colacc[b][4 * h + 2] & 0x7FFF7FFFu, w3 = colacc[b][4 * h + 3] & 0x7FFF7FFFu;
+                    if (w0 | w1 | w2 | w3) red_max_bf16x8(dst + 4 * h, w0, w1, w2, w3);
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) colacc[b][k] = 0u;
+            }
+        } else if (p.amax_col) {
 #pragma unroll
             for (int b = 0; b < BT; ++b) {
                 if (!valid[b]) continue;

@@ -165,6 +165,25 @@ def test_repeated_calls_reuse_buffers(orc):
         compare(to_np(out), orc.quantize(x), label=f"reuse {seed}")
 
 
+@pytest.mark.parametrize("shape", [(1040, 1056), (64, 16400)], ids=["row_pass", "tile_path"])
+def test_timed_cast_matches_plain_cast(shape):
+    """The measurement hook records its events around the three launches and leaves
+    every output bit as the plain call writes it (both kernel routes)."""
+    x = inputs.random_shape(21, *shape, "wide").cuda()
+    buf_a = torch.full((1,), 2.0, device="cuda")
+    buf_b = buf_a.clone()
+    plain = nv.quantize(x, absmax=buf_a, decay=0.9)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(nv.CAST_LAUNCHES + 1)]
+    for e in evs:
+        e.record()
+    timed = nv.quantize_timed(x, evs, absmax=buf_b, decay=0.9)
+    torch.cuda.synchronize()
+    compare(to_np(timed), to_np(plain), label="timed vs plain")
+    assert buf_a.cpu().numpy().view(np.uint32)[0] == buf_b.cpu().numpy().view(np.uint32)[0]
+    for i in range(nv.CAST_LAUNCHES):
+        assert evs[i].elapsed_time(evs[i + 1]) > 0.0
+
+
 def test_update_absmax(orc):
     rng = np.random.default_rng(14)
     for n in (0, 1, 1000, 1 << 20):
