@@ -134,7 +134,7 @@ cudaError_t launch_zero(cudaStream_t stream, const ZeroParams& z)
     int64_t total = 0;
     for (int k = 0; k < 4; ++k) total += z.ptr[k] ? z.n4[k] : 0;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(148, (total + kThreads - 1) / kThreads));
-    return launch(pass0_zero, grid, 0, stream, z, false);
+    return launch(pass0_zero, grid, 0, stream, z, true);
 }
 
 // The geometry and group tables of a call (offsets already validated).

@@ -114,6 +114,8 @@ template <int MAXG>
 __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant__ ColParams<MAXG> p)
 {
     // per warp: codes [column][16 chunks of 8 bytes] (swizzled), then scales [column][16]
+    // The next cast's zeroing kernel may take its place early; it waits for this grid.
+    griddep_launch_dependents();
     extern __shared__ __align__(16) uint8_t col_stage[];
     __shared__ uint32_t rcp_tab[8];
     init_rcp_table(rcp_tab);

@@ -24,8 +24,12 @@ struct ZeroParams {
     uint32_t* err;     // error word to clear (may be null)
 };
 
+// Launched as a programmatic dependent of whatever precedes the cast on the stream: it
+// waits for that grid (and its memory) before anything else, and only then lets the
+// cast's next kernel start, which reads x without waiting itself.
 __global__ void __launch_bounds__(kThreads) pass0_zero(const __grid_constant__ ZeroParams p)
 {
+    griddep_wait();
     griddep_launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
