@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_quantize_weight_2d.restype = ctypes.c_int
         _lib.oracle_e4m3_array.argtypes, _lib.oracle_e4m3_array.restype = [P, I64, P], None
         _lib.oracle_e2m1_array.argtypes, _lib.oracle_e2m1_array.restype = [P, I64, P], None
+        _lib.oracle_f32_to_bf16_array.argtypes, _lib.oracle_f32_to_bf16_array.restype = [P, I64, P], None
+        _lib.oracle_dequantize_rows.argtypes = [P, P, P, I64, I64, P]
+        _lib.oracle_dequantize_rows.restype = ctypes.c_int
     return _lib
 
 
@@ -239,3 +242,46 @@ def dequantize_rows(q, sf, amax):
     scale = sft[np.asarray(sf, np.uint8)].repeat(16, axis=1)
     senc = np.array([s_enc(float(a)) for a in np.asarray(amax, np.float32)], np.float64)[:, None]
     return vals * scale / senc
+
+
+def f32_to_bf16(v) -> np.ndarray:
+    """uint16 bits of the nearest bf16 to each binary32 value (ties to even)."""
+    a = np.ascontiguousarray(np.asarray(v, np.float32))
+    out = np.zeros(a.shape, np.uint16)
+    lib().oracle_f32_to_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def dequantize(q, sf, amax) -> np.ndarray:
+    """oracle_dequantize_rows: bf16 bits [M, K] of rowwise-layout NVFP4 data
+    (q [M, K/2], sf [M, K/16], amax [M]); columnwise data [K, M/2], [K, M/16], [K]
+    give X^T."""
+    qa = np.ascontiguousarray(np.asarray(q, np.uint8))
+    M, half = qa.shape
+    K = 2 * half
+    sfa = np.ascontiguousarray(np.asarray(sf, np.uint8).reshape(M, K // 16))
+    am = np.ascontiguousarray(np.asarray(amax, np.float32).reshape(M))
+    out = np.zeros((M, K), np.uint16)
+    if lib().oracle_dequantize_rows(_ptr(qa), _ptr(sfa), _ptr(am), M, K, _ptr(out)) != 0:
+        raise ValueError(f"oracle_dequantize_rows: bad shape {M}x{K}")
+    return out
+
+
+def requantize_colwise(q_row, sf_row, amax_row, offsets=None, absmax=None, decay: float = 0.0) -> dict:
+    """Columnwise requantization of rowwise-quantized data: the columnwise cast (per
+    token group when offsets are given) of X' = dequantize(q_row, sf_row, amax_row),
+    the NVFP4 per-token analog of the "dequantize, then columnwise-only requantize"
+    step of TransformerEngine PR #3244 (flowchart). It adds no arithmetic of its own:
+    both steps are the oracle's dequantize and cast."""
+    xd = dequantize(q_row, sf_row, amax_row)
+    M = xd.shape[0]
+    off = [0, M] if offsets is None else offsets
+    out = quantize_grouped(xd.view(np.uint16), off, flags=COLWISE, absmax=absmax, decay=decay)
+    res = {k: out[k] for k in ("q_col", "sf_col", "amax_col")}
+    if offsets is None:
+        res["q_col"] = res["q_col"].reshape(xd.shape[1], M // 2)
+        res["sf_col"] = res["sf_col"].reshape(xd.shape[1], M // 16)
+        res["amax_col"] = res["amax_col"].reshape(-1)
+    if "absmax" in out:
+        res["absmax"] = out["absmax"]
+    return res

@@ -349,6 +349,54 @@ int oracle_quantize_weight_2d(const uint16_t* w, int64_t N, int64_t K,
     return 0;
 }
 
+/* --------------------------------------------------------- dequantization */
+
+/* Nearest bf16 to a finite binary32 f, ties to the even significand: the two bf16
+ * neighbours of |f| (its truncation and the next magnitude up) are compared in
+ * double, where both distances are exact. */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    const uint16_t lo = (uint16_t)(u >> 16);   /* truncation toward zero, same sign */
+    if ((u & 0xFFFFu) == 0) return lo;         /* exactly representable */
+    const uint16_t hi = (uint16_t)(lo + 1);    /* next magnitude away from zero */
+    const double a = fabs((double)f);
+    const double dl = a - fabs((double)oracle_bf16_to_f32(lo));
+    const double dh = fabs((double)oracle_bf16_to_f32(hi)) - a;
+    if (dl < dh) return lo;
+    if (dh < dl) return hi;
+    return (lo & 1) ? hi : lo;
+}
+
+/* Dequantization of rowwise-layout NVFP4 data, the inverse of the cast (the pages
+ * store fp32 "scale_inv" factors beside the block scales, TransformerEngine PR #3296;
+ * PR #3244's flow dequantizes rowwise data before requantizing it columnwise). The
+ * reading taken: with the decode scale S_dec = RN(amax / 2688) of the row,
+ *     x'[r][16b + j] = bf16_rn( RN( (val(q) * float(sf[r][b])) * S_dec ) ),
+ * where val(q) * float(sf) is exact in binary32 (at most 2 + 4 significant bits).
+ * q: [M, K/2] (element 2j in the low nibble), sf: [M, K/16], amax: [M]; out: bf16
+ * [M, K]. The columnwise data [K, M/2], [K, M/16], [K] give X^T the same way. */
+int oracle_dequantize_rows(const uint8_t* q, const uint8_t* sf, const float* amax, int64_t M, int64_t K,
+                           uint16_t* out)
+{
+    if (!shape_ok(M, K)) return -1;
+    for (int64_t r = 0; r < M; ++r) {
+        const float sdec = amax[r] / 2688.0f;
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const float s = oracle_e4m3_decode(sf[r * (K / 16) + b]);
+            for (int j = 0; j < 16; ++j) {
+                const uint8_t byte = q[r * (K / 2) + 8 * b + j / 2];
+                const uint8_t code = (j & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+                const float t = oracle_e2m1_decode(code) * s; /* exact */
+                const float y = t * sdec;
+                out[r * K + 16 * b + j] = oracle_f32_to_bf16(y);
+            }
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------ array forms (for sweeps) */
 
 void oracle_e4m3_array(const float* v, int64_t n, uint8_t* out)
@@ -359,4 +407,9 @@ void oracle_e4m3_array(const float* v, int64_t n, uint8_t* out)
 void oracle_e2m1_array(const float* y, int64_t n, uint8_t* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1(y[i]);
+}
+
+void oracle_f32_to_bf16_array(const float* v, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16(v[i]);
 }
