@@ -343,6 +343,82 @@ def run_gpu(args, dist: Dist) -> dict | None:
 
 # ------------------------------------------------------------ oracle arm
 
+def op_bytes(op: str, m: int, k: int) -> int:
+    """Algorithmic bytes of the secondary ops. Dequantize: rowwise codes, scales and
+    amax in, bf16 out. Columnwise requantize: rowwise data in, columnwise data out
+    (the least any implementation must move)."""
+    rowdata = m * k // 2 + m * k // 16 + 4 * m
+    if op == "dequant":
+        return rowdata + 2 * m * k
+    return rowdata + m * k // 2 + m * k // 16 + 4 * k
+
+
+def run_gpu_op(args, dist: Dist, op: str) -> dict | None:
+    """Device time of nvfp4pt_dequantize or nvfp4pt_requantize_colwise on the rowwise
+    outputs of the headline activation (two rotating input sets)."""
+    import torch
+
+    import precision_quantization_row_b200 as nv
+    from precision_quantization_row_b200 import build, inputs
+
+    build.build()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    stream = torch.cuda.current_stream(dev)
+    m, k = args.rows, args.cols
+    x = inputs.llm(M=m, K=k).to(dev)
+    srcs = [nv.quantize(x, flags=nv.ROWWISE), nv.quantize(x.neg(), flags=nv.ROWWISE)]
+    del x
+    if op == "dequant":
+        outs = [torch.empty((m, k), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+
+        def step(i):
+            s = srcs[i & 1]
+            nv.dequantize(s["q_row"], s["sf_row"], s["amax_row"], out=outs[i & 1], stream=stream)
+        launches = 1
+    else:
+        ws = torch.empty(nv.requantize_workspace_bytes(m, k, 1), dtype=torch.uint8, device=dev)
+        outs = [None, None]
+
+        def step(i):
+            s = srcs[i & 1]
+            outs[i & 1] = nv.requantize_colwise(s["q_row"], s["sf_row"], s["amax_row"], out=outs[i & 1],
+                                                workspace=ws, stream=stream)
+        launches = 1 + nv.CAST_LAUNCHES
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run():
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1) / 1e3
+
+    with ClockSampler(dev.index) as clk:
+        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    if dist.rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    per = secs / args.steps
+    achieved = op_bytes(op, m, k) / per / 1e9
+    name = {"dequant": "NVFP4 rowwise dequantize to bf16", "requant": "NVFP4 rowwise -> columnwise requantize"}[op]
+    return {
+        "metric": f"{name}: elems/s, achieved HBM GB/s", "value": float(m) * k * args.steps * dist.world / secs,
+        "unit": "elem/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4->bf16" if op == "dequant" else "nvfp4->nvfp4 (via bf16)", "data": "synthetic",
+        "config": {"workload": f"{op}_rowwise_{m}x{k}", "rows": m, "cols": k,
+                   "l2": "two rotating input sets and outputs"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_kind, "algorithmic_bytes_per_call": op_bytes(op, m, k)},
+        "gpu_launches": launches * args.steps, "clocks": clk.summary(),
+    }
+
+
 def oracle_sample_rate(rows: int) -> tuple[float, str]:
     """elems/s of the oracle's full row+col cast (with the absmax update) of the
     first `rows` rows of the benchmark matrix, single-threaded."""
@@ -403,6 +479,8 @@ def main(argv=None):
     ap.add_argument("--cols", type=int, default=8192, help="columns of the activation (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--op", choices=["cast", "dequant", "requant"], default="cast",
+                    help="cast: the per-token cast (the headline); dequant / requant: the secondary ops")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -412,6 +490,14 @@ def main(argv=None):
             print(json.dumps(line), flush=True)
         return
     dist = Dist(args.gpus)
+    if args.op != "cast":
+        try:
+            line = run_gpu_op(args, dist, args.op)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+        finally:
+            dist.close()
+        return
     try:
         line = run_gpu(args, dist)
         if line is not None and dist.world == 1 and not args.no_cpu_baseline:

@@ -149,6 +149,52 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w_bf16, int64_
                                           void* workspace, cudaStream_t stream);
 
 /*
+ * nvfp4pt_dequantize -- rowwise-layout NVFP4 data back to bf16. The pages keep fp32
+ * "scale_inv" factors beside the block scales (PR #3296, title and Description) and
+ * dequantize rowwise data before requantizing it (PR #3244, flowchart: "Dequantize",
+ * then "Columnwise-only requantize"); the exact formula is not printed. Reading taken:
+ * with the decode scale S_dec = RN(amax[r] / 2688) of row r,
+ *     out[r][16b + j] = bf16_rn( RN( (val(q) * float(sf[r][b])) * S_dec ) ),
+ * val(q) * float(sf) being exact in binary32. An amax of 0 gives signed zeros.
+ *
+ * q        uint8 [rows, cols/2]  codes, element 2j in the low nibble of byte j.
+ * sf       uint8 [rows, cols/16] E4M3 block scales.
+ * amax     fp32  [rows]          the rows' amax (as the cast wrote it).
+ * out_bf16 bf16  [rows, cols]    written in full.
+ * Columnwise data (q_col [cols, rows/2], sf_col [cols, rows/16], amax_col [cols])
+ * passed with rows and cols swapped give X^T. Same conventions as the casts (device
+ * pointers, 16-byte alignment, sizes multiples of 16, asynchronous on `stream`); no
+ * workspace.
+ */
+NVFP4PT_API nvfp4pt_status nvfp4pt_dequantize(const uint8_t* q, const uint8_t* sf, const float* amax,
+                                              int64_t rows, int64_t cols, void* out_bf16, cudaStream_t stream);
+
+/* Workspace bytes of nvfp4pt_requantize_colwise: the dequantized bf16 matrix
+ * (rows * cols * 2, rounded up to 256) plus nvfp4pt_workspace_bytes(rows, cols, num_groups). */
+NVFP4PT_API size_t nvfp4pt_requantize_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
+
+/*
+ * nvfp4pt_requantize_colwise -- columnwise NVFP4 data made from rowwise NVFP4 data
+ * (the per-token NVFP4 analog of PR #3244's "dequant + requant with col-wise to save
+ * for backward", Description and flowchart): the columnwise cast, per token group,
+ * of X' = nvfp4pt_dequantize(q_row, sf_row, amax_row).
+ *
+ * offsets_host  NULL (one group: outputs as nvfp4pt_quantize's columnwise ones) or
+ *               num_groups+1 host row offsets as in nvfp4pt_quantize_grouped.
+ * q_col, sf_col, amax_col, absmax_bufs, decay: as in nvfp4pt_quantize_grouped's
+ *               columnwise direction (absmax_bufs NULL or [groups]; Observed = the
+ *               group's max |x'|).
+ * workspace     nvfp4pt_requantize_workspace_bytes(rows, cols, groups) bytes.
+ * Errors as in nvfp4pt_quantize_grouped, reported before anything is launched.
+ */
+NVFP4PT_API nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, const uint8_t* sf_row,
+                                                      const float* amax_row, int64_t rows, int64_t cols,
+                                                      const int64_t* offsets_host, int num_groups,
+                                                      uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                                      float* absmax_bufs, float decay, void* workspace,
+                                                      cudaStream_t stream);
+
+/*
  * nvfp4pt_update_absmax -- the running-buffer step alone (PR #3296, Description):
  * *absmax_buf = max(RN(*absmax_buf * decay), max_i amax_vec[i]); n may be 0
  * (Observed = 0). Both pointers are device pointers; amax_vec holds n non-negative

@@ -35,7 +35,8 @@ EXPORTS = (
     "nvfp4pt_quantize_weight_2d", "nvfp4pt_update_absmax", "nvfp4pt_workspace_error",
     "nvfp4pt_probe_transitions", "nvfp4pt_probe_pairs", "nvfp4pt_probe_e4m3_decode", "nvfp4pt_probe_div6",
     "nvfp4pt_probe_e4m3_div", "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_probe_pair_scales",
-    "nvfp4pt_quantize_timed",
+    "nvfp4pt_quantize_timed", "nvfp4pt_dequantize", "nvfp4pt_requantize_workspace_bytes",
+    "nvfp4pt_requantize_colwise",
 )
 
 
@@ -72,8 +73,12 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_quantize_grouped_noalloc.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, F, P]
         L.nvfp4pt_probe_pair_scales.argtypes = [I, I, ctypes.c_uint32, P, P]
         L.nvfp4pt_quantize_timed.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, F, P, P, P]
+        L.nvfp4pt_dequantize.argtypes = [P, P, P, I64, I64, P, P]
+        L.nvfp4pt_requantize_workspace_bytes.argtypes = [I64, I64, I]
+        L.nvfp4pt_requantize_colwise.argtypes = [P, P, P, I64, I64, P, I, P, P, P, P, F, P, P]
         for name in EXPORTS[2:]:
             getattr(L, name).restype = I
+        L.nvfp4pt_requantize_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -162,6 +167,57 @@ def quantize_timed(x: torch.Tensor, events, flags: int = ROWWISE | COLWISE, absm
         _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("amax_col")), _ptr(absmax),
         ctypes.c_float(decay), _ptr(ws), _stream(stream, x.device), evs)
     _check("nvfp4pt_quantize_timed", st)
+    return out
+
+
+def dequantize(q: torch.Tensor, sf: torch.Tensor, amax: torch.Tensor, out: torch.Tensor | None = None,
+               stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """nvfp4pt_dequantize: rowwise-layout NVFP4 data (q uint8 [rows, cols/2], sf uint8
+    [rows, cols/16], amax fp32 [rows]) back to bf16 [rows, cols]."""
+    for t, n in ((q, "q"), (sf, "sf"), (amax, "amax")):
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+    rows, half = q.shape
+    cols = 2 * half
+    out = torch.empty((rows, cols), dtype=torch.bfloat16, device=q.device) if out is None else out
+    st = lib().nvfp4pt_dequantize(_ptr(q), _ptr(sf), _ptr(amax), rows, cols, _ptr(out), _stream(stream, q.device))
+    _check("nvfp4pt_dequantize", st)
+    return out
+
+
+def requantize_workspace_bytes(rows: int, cols: int, groups: int = 1) -> int:
+    return int(lib().nvfp4pt_requantize_workspace_bytes(rows, cols, groups))
+
+
+def requantize_colwise(q_row: torch.Tensor, sf_row: torch.Tensor, amax_row: torch.Tensor, offsets=None,
+                       absmax: torch.Tensor | None = None, decay: float = 0.0, out: dict | None = None,
+                       workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> dict:
+    """nvfp4pt_requantize_colwise: the columnwise outputs (q_col, sf_col, amax_col) of the
+    cast of the dequantized rowwise data; offsets: None or the host row offsets of the
+    token groups."""
+    for t, n in ((q_row, "q_row"), (sf_row, "sf_row"), (amax_row, "amax_row")):
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+    rows, half = q_row.shape
+    cols = 2 * half
+    G = 1 if offsets is None else len(offsets) - 1
+    if out is None:
+        dev = q_row.device
+        if offsets is None:
+            out = {"q_col": torch.empty((cols, rows // 2), dtype=torch.uint8, device=dev),
+                   "sf_col": torch.empty((cols, rows // 16), dtype=torch.uint8, device=dev),
+                   "amax_col": torch.empty(cols, dtype=torch.float32, device=dev)}
+        else:
+            out = {"q_col": torch.empty(cols * rows // 2, dtype=torch.uint8, device=dev),
+                   "sf_col": torch.empty(cols * rows // 16, dtype=torch.uint8, device=dev),
+                   "amax_col": torch.empty((G, cols), dtype=torch.float32, device=dev)}
+    if workspace is None:
+        workspace = torch.empty(requantize_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=q_row.device)
+    off = None if offsets is None else (ctypes.c_int64 * len(offsets))(*[int(o) for o in offsets])
+    st = lib().nvfp4pt_requantize_colwise(
+        _ptr(q_row), _ptr(sf_row), _ptr(amax_row), rows, cols, off, G, _ptr(out["q_col"]), _ptr(out["sf_col"]),
+        _ptr(out["amax_col"]), _ptr(absmax), ctypes.c_float(decay), _ptr(workspace), _stream(stream, q_row.device))
+    _check("nvfp4pt_requantize_colwise", st)
     return out
 
 

@@ -13,6 +13,7 @@
 #include "nvfp4pt_kernels.cuh"
 #include "nvfp4pt_rowpass.cuh"
 #include "nvfp4pt_colpass.cuh"
+#include "nvfp4pt_dequant.cuh"
 
 using namespace nvfp4pt;
 
@@ -312,6 +313,23 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
     return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 
+cudaError_t launch_dequant(const uint8_t* q, const uint8_t* sf, const float* amax, int64_t rows, int64_t cols,
+                           uint16_t* out, int sm_count, cudaStream_t stream)
+{
+    DequantParams d;
+    d.q = q;
+    d.sf = sf;
+    d.amax = amax;
+    d.out = out;
+    d.rows = rows;
+    d.cols = cols;
+    const int grid = (int)std::min<int64_t>(rows, 8 * (int64_t)sm_count);
+    dequant_rows_kernel<<<grid, 256, 0, stream>>>(d);
+    return cudaGetLastError();
+}
+
+int64_t requant_bf16_bytes(int64_t rows, int64_t cols) { return align256(rows * cols * 2); }
+
 }  // namespace
 
 extern "C" {
@@ -449,6 +467,58 @@ nvfp4pt_status nvfp4pt_workspace_error(const void* workspace, uint32_t* word, cu
         return NVFP4PT_ERR_CUDA;
     if (word) *word = w;
     return w ? NVFP4PT_ERR_DEVICE : NVFP4PT_OK;
+}
+
+nvfp4pt_status nvfp4pt_dequantize(const uint8_t* q, const uint8_t* sf, const float* amax, int64_t rows, int64_t cols,
+                                  void* out_bf16, cudaStream_t stream)
+{
+    if (!q || !sf || !amax || !out_bf16) return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = check_shape(rows, cols);
+    if (st != NVFP4PT_OK) return st;
+    if (!aligned16(q) || !aligned16(sf) || !aligned16(amax) || !aligned16(out_bf16)) return NVFP4PT_ERR_ALIGN;
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4PT_OK) return st;
+    return launch_dequant(q, sf, amax, rows, cols, static_cast<uint16_t*>(out_bf16), dev->sm_count, stream) ==
+                   cudaSuccess
+               ? NVFP4PT_OK
+               : NVFP4PT_ERR_CUDA;
+}
+
+size_t nvfp4pt_requantize_workspace_bytes(int64_t rows, int64_t cols, int num_groups)
+{
+    const int64_t r = rows < 0 ? 0 : rows, c = cols < 0 ? 0 : cols;
+    return (size_t)requant_bf16_bytes(r, c) + nvfp4pt_workspace_bytes(rows, cols, num_groups);
+}
+
+nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, const uint8_t* sf_row, const float* amax_row,
+                                          int64_t rows, int64_t cols, const int64_t* offsets_host, int num_groups,
+                                          uint8_t* q_col, uint8_t* sf_col, float* amax_col, float* absmax_bufs,
+                                          float decay, void* workspace, cudaStream_t stream)
+{
+    if (!q_row || !sf_row || !amax_row || !q_col || !sf_col || !amax_col || !workspace) return NVFP4PT_ERR_NULL;
+    nvfp4pt_status st = check_shape(rows, cols);
+    if (st != NVFP4PT_OK) return st;
+    if (!aligned16(q_row) || !aligned16(sf_row) || !aligned16(amax_row) || !aligned16(q_col) || !aligned16(sf_col) ||
+        !aligned16(amax_col) || !aligned16(static_cast<uint8_t*>(workspace)) || (absmax_bufs && !aligned16(absmax_bufs)))
+        return NVFP4PT_ERR_ALIGN;
+    const int64_t one[2] = {0, rows};
+    const int64_t* off = offsets_host ? offsets_host : one;
+    const int G = offsets_host ? num_groups : 1;
+    if (G < 1 || G > NVFP4PT_MAX_GROUPS || off[0] != 0 || off[G] != rows) return NVFP4PT_ERR_GROUPS;
+    for (int g = 0; g < G; ++g)
+        if (off[g + 1] < off[g] || off[g] % 16) return NVFP4PT_ERR_GROUPS;
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4PT_OK) return st;
+    // X' (bf16) in the workspace, then the columnwise cast of X' with the rest of it
+    uint16_t* xd = static_cast<uint16_t*>(workspace);
+    void* ws = static_cast<uint8_t*>(workspace) + requant_bf16_bytes(rows, cols);
+    if (launch_dequant(q_row, sf_row, amax_row, rows, cols, xd, dev->sm_count, stream) != cudaSuccess)
+        return NVFP4PT_ERR_CUDA;
+    if (G == 1)
+        return run_cast<1>(xd, rows, cols, off, 1, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col, sf_col,
+                           amax_col, absmax_bufs, decay, false, ws, stream);
+    return run_cast<kMaxGroups>(xd, rows, cols, off, G, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col, sf_col,
+                                amax_col, absmax_bufs, decay, false, ws, stream);
 }
 
 }  // extern "C"

@@ -1,0 +1,87 @@
+// Dequantization of rowwise-layout NVFP4 data (sm_100a): codes [rows, cols/2], E4M3
+// block scales [rows, cols/16] and row amaxes [rows] back to bf16 [rows, cols]:
+//     x' = bf16_rn( RN( (val(q) * float(sf)) * RN(amax / 2688) ) ),
+// the inverse of the cast with the decode scale amax/2688 (the "scale_inv" factor
+// the TransformerEngine pages store beside the block scales). val(q) * float(sf) is
+// exact in binary32. Columnwise data ([cols, rows/2], ...) give X^T the same way.
+//
+// CTAs take rows (grid-strided), threads the 16-element blocks of a row: 8 code bytes
+// and one scale byte in, 32 bytes out; the row's decode scale once per row and
+// thread. HBM-bound: 0.5625 B read and 2 B written per element.
+#pragma once
+
+#include "nvfp4pt_device.cuh"
+
+namespace nvfp4pt {
+
+struct DequantParams {
+    const uint8_t* q;
+    const uint8_t* sf;
+    const float* amax;
+    uint16_t* out;
+    int64_t rows;
+    int64_t cols;
+};
+
+// The E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are bf16 values: high bytes
+// 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0. One byte permute per
+// table picks the bytes of four codes at once (selector nibble = the code's 3-bit
+// magnitude index); the sign goes to bit 15.
+__device__ __forceinline__ void e2m1x4_to_bf16(uint32_t codes4, uint32_t& w01, uint32_t& w23)
+{
+    const uint32_t sel = codes4 & 0x7777u;   // nibble i: magnitude index of element i
+    const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);   // high byte of element i -> byte i
+    const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);   // low byte of element i -> byte i
+    // element i's bf16 = hi byte i : lo byte i; elements 0,1 -> w01 (0 in the low half)
+    w01 = __byte_perm(lo, hi, 0x5140);
+    w23 = __byte_perm(lo, hi, 0x7362);
+    // signs: code bit 3 of element i -> bit 15 of its half
+    const uint32_t s = codes4 & 0x8888u;
+    w01 |= ((s & 0x8u) << 12) | ((s & 0x80u) << 24);
+    w23 |= ((s & 0x800u) << 4) | ((s & 0x8000u) << 16);
+}
+
+// (bf16(RN(a.lo * m)), bf16(RN(a.hi * m))) for the two exact products in a (binary32
+// pair) and the decode scale m, as one bf16x2 word (first element in the low half).
+__device__ __forceinline__ uint32_t scale_to_bf16x2(float t0, float t1, float m)
+{
+    float y0, y1;
+    mul2(y0, y1, t0, t1, m);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y1), "f"(y0));
+    return r;
+}
+
+__global__ void __launch_bounds__(256) dequant_rows_kernel(const __grid_constant__ DequantParams p)
+{
+    const int64_t bpr = p.cols / 16;   // blocks per row
+    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+        const float m = __fdiv_rn(p.amax[row], 2688.0f);   // decode scale of the row
+        for (int64_t j = threadIdx.x; j < bpr; j += blockDim.x) {
+            const int64_t b = row * bpr + j;
+            const uint2 c8 = *reinterpret_cast<const uint2*>(p.q + 8 * b);   // 16 codes, element 2i low nibble
+            float s, s_unused;
+            e4m3x2_decode(p.sf[b], s, s_unused);
+            uint32_t out[8];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                // codes of elements 4h..4h+3: byte pair h of the 8 code bytes
+                const uint32_t w = (h < 2) ? c8.x : c8.y;
+                const uint32_t codes4 = (w >> (16 * (h & 1))) & 0xFFFFu;
+                uint32_t b01, b23;
+                e2m1x4_to_bf16(codes4, b01, b23);
+                // val * float(sf): exact, from the bf16 magnitudes
+                float t0, t1, t2, t3;
+                mul2(t0, t1, bf16_lo(b01), bf16_hi(b01), s);
+                mul2(t2, t3, bf16_lo(b23), bf16_hi(b23), s);
+                out[2 * h] = scale_to_bf16x2(t0, t1, m);
+                out[2 * h + 1] = scale_to_bf16x2(t2, t3, m);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.out + 16 * b);
+            dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+            dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        }
+    }
+}
+
+}  // namespace nvfp4pt

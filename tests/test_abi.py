@@ -118,6 +118,34 @@ def test_weight_and_absmax_rejections(L):
     assert L.nvfp4pt_workspace_error(None, None, None) == 1
 
 
+def test_dequant_and_requant_rejections(L):
+    h = _Host()
+    P = h.p
+    d = L.nvfp4pt_dequantize
+    assert d(None, P(), P(), 16, 16, P(), None) == 1
+    assert d(P(), P(), P(), 16, 16, None, None) == 1
+    assert d(P(), P(), P(), 16, 24, P(), None) == 2
+    assert d(P(), P(8), P(), 16, 16, P(), None) == 3
+    assert d(P(), P(), P(), 16, 16, P(4), None) == 3
+    assert L.nvfp4pt_requantize_workspace_bytes(16, 16, 1) >= 16 * 16 * 2 + L.nvfp4pt_workspace_bytes(16, 16, 1)
+
+    def r(*args, offs=None, G=1, rows=64, ws=None):
+        arr = None if offs is None else (ctypes.c_int64 * len(offs))(*offs)
+        a = list(args) if args else [P()] * 3
+        return L.nvfp4pt_requantize_colwise(*a, rows, 32, arr, G, P(), P(), P(), None, F0,
+                                            P() if ws is None else ws, None)
+
+    assert r(None, P(), P()) == 1
+    assert L.nvfp4pt_requantize_colwise(P(), P(), P(), 64, 32, None, 1, P(), P(), P(), None, F0, None, None) == 1
+    assert L.nvfp4pt_requantize_colwise(P(), P(), P(), 64, 20, None, 1, P(), P(), P(), None, F0, P(), None) == 2
+    assert r(P(), P(), P(2)) == 3
+    assert r(offs=[0, 8, 64], G=2) == 4
+    assert r(offs=[0, 64], G=0) == 4
+    # valid (ungrouped and grouped) pass validation and fail only at the device step here
+    assert r() in (5, 6)
+    assert r(offs=[0, 0, 32, 64], G=3) in (5, 6)
+
+
 def test_probe_rejections(L):
     h = _Host()
     P = h.p

@@ -1,0 +1,85 @@
+"""GPU parity of the dequantization and the columnwise requantization against the
+oracle, bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import precision_quantization_row_b200 as nv
+from precision_quantization_row_b200 import inputs
+from parity_util import compare, to_np
+
+pytestmark = pytest.mark.gpu
+
+FINITE_SF = [c for c in range(256) if c not in (0x7F, 0xFF)]
+
+
+def _random_rows(seed, rows, cols):
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
+    sf = rng.choice(FINITE_SF, (rows, cols // 16)).astype(np.uint8)
+    amax = (rng.standard_normal(rows) * 10.0 ** rng.integers(-30, 30, rows)).astype(np.float32)
+    amax = np.abs(amax)
+    special = np.array([0.0, 2688.0, 2688.0 * 2 ** -20, 2688.0 * 2 ** 40, 3.3e38, 1e-38, 5e-39, 1.0], np.float32)
+    amax[: min(rows, special.size)] = special[: min(rows, special.size)]
+    return q, sf, amax
+
+
+@pytest.mark.parametrize("shape", [(16, 16), (48, 80), (272, 144), (1040, 1056), (4096, 16), (16, 4096)],
+                         ids=lambda s: f"{s[0]}x{s[1]}")
+def test_dequant_random_codes(orc, shape):
+    q, sf, amax = _random_rows(sum(shape), *shape)
+    got = nv.dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), torch.from_numpy(amax).cuda())
+    want = orc.dequantize(q, sf, amax)
+    g = got.cpu().view(torch.int16).numpy().view(np.uint16)
+    bad = np.argwhere(g != want)
+    assert bad.size == 0, f"{bad.shape[0]} mismatches, first {bad[:3].tolist()}"
+
+
+@pytest.mark.parametrize("kind", ["normal", "wide", "tiny", "signed_zero"])
+def test_dequant_of_cast_outputs(orc, kind):
+    x = inputs.random_shape(61, 512, 768, kind).cuda()
+    out = nv.quantize(x, flags=nv.ROWWISE)
+    got = nv.dequantize(out["q_row"], out["sf_row"], out["amax_row"])
+    want = orc.dequantize(out["q_row"].cpu().numpy(), out["sf_row"].cpu().numpy(), out["amax_row"].cpu().numpy())
+    assert np.array_equal(got.cpu().view(torch.int16).numpy().view(np.uint16), want)
+
+
+def _rows_of(x):
+    out = nv.quantize(x.cuda(), flags=nv.ROWWISE)
+    return out["q_row"], out["sf_row"], out["amax_row"]
+
+
+@pytest.mark.parametrize("shape", [(256, 512), (1040, 1056), (4096, 4096)], ids=lambda s: f"{s[0]}x{s[1]}")
+def test_requant_colwise(orc, shape):
+    x = inputs.random_shape(62, *shape, "wide")
+    q, sf, a = _rows_of(x)
+    buf = torch.full((1,), 5.0, device="cuda")
+    got = nv.requantize_colwise(q, sf, a, absmax=buf, decay=0.75)
+    want = orc.requantize_colwise(q.cpu().numpy(), sf.cpu().numpy(), a.cpu().numpy(),
+                                  absmax=np.array([5.0], np.float32), decay=0.75)
+    compare(to_np(got), {k: want[k] for k in ("q_col", "sf_col", "amax_col")}, label=f"requant {shape}")
+    assert np.float32(buf.item()).view(np.uint32) == np.float32(want["absmax"][0]).view(np.uint32)
+
+
+def test_requant_grouped(orc):
+    x = inputs.random_shape(63, 400, 272, "normal")
+    offsets = [0, 0, 48, 48, 320, 400]
+    q, sf, a = _rows_of(x)
+    bufs = torch.arange(5, dtype=torch.float32, device="cuda")
+    got = nv.requantize_colwise(q, sf, a, offsets=offsets, absmax=bufs, decay=0.5)
+    want = orc.requantize_colwise(q.cpu().numpy(), sf.cpu().numpy(), a.cpu().numpy(), offsets=offsets,
+                                  absmax=np.arange(5, dtype=np.float32), decay=0.5)
+    compare(to_np(got), {k: want[k] for k in ("q_col", "sf_col", "amax_col")}, label="grouped requant")
+    assert np.array_equal(bufs.cpu().numpy().view(np.uint32), want["absmax"].view(np.uint32))
+
+
+def test_requant_of_lossless_rows_equals_direct_cast():
+    """Rows whose cast is lossless: requantizing their rowwise data on the GPU gives the
+    GPU's direct columnwise cast of the matrix itself."""
+    from test_oracle_dequant import _lossless_matrix
+    x = _lossless_matrix(np.random.default_rng(64), 256, 320).cuda()
+    q, sf, a = _rows_of(x)
+    got = nv.requantize_colwise(q, sf, a)
+    direct = nv.quantize(x, flags=nv.COLWISE)
+    for k in ("q_col", "sf_col", "amax_col"):
+        assert torch.equal(got[k].reshape(-1), direct[k].reshape(-1)), k
