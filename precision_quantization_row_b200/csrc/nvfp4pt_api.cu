@@ -57,7 +57,8 @@ nvfp4pt_status device_state(DeviceState** out)
                     cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
             }
-            const void* colpasses[] = {(const void*)colpass<1>, (const void*)colpass<kMaxGroups>};
+            const void* colpasses[] = {(const void*)colpass<1, false>, (const void*)colpass<kMaxGroups, false>,
+                                       (const void*)colpass<1, true>, (const void*)colpass<kMaxGroups, true>};
             for (const void* f : colpasses) {
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColPass) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
@@ -180,21 +181,30 @@ RowShape row_shape(int64_t cols)
     return r;
 }
 
-template <int MAXG>
+template <int MAXG, bool NV>
 cudaError_t launch_rowpass(const RowShape& rs, const RowParams<MAXG>& rp, cudaStream_t stream)
 {
     const int grid = rp.num_ctas;
-    if (rs.bt == 2) return launch(rowpass<MAXG, 2, 2>, grid, 0, stream, rp, true, kRowThreads);
-    if (rs.S == 4) return launch(rowpass<MAXG, 1, 4>, grid, 0, stream, rp, true, kRowThreads);
-    if (rs.S == 2) return launch(rowpass<MAXG, 1, 2>, grid, 0, stream, rp, true, kRowThreads);
-    return launch(rowpass<MAXG, 1, 1>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.bt == 2) return launch(rowpass<MAXG, 2, 2, NV>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.S == 4) return launch(rowpass<MAXG, 1, 4, NV>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.S == 2) return launch(rowpass<MAXG, 1, 2, NV>, grid, 0, stream, rp, true, kRowThreads);
+    return launch(rowpass<MAXG, 1, 1, NV>, grid, 0, stream, rp, true, kRowThreads);
 }
+
+// NVFP4 rowwise data as the cast's source (the requantization): codes, scales, row
+// amaxes, and room for the rows' decode scales.
+struct NvSource {
+    const uint8_t* q;
+    const uint8_t* sf;
+    const float* amax;
+    float* dscale;
+};
 
 template <int MAXG>
 nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t* off, int G, int flags,
                         uint8_t* q_row, uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col,
                         float* amax_col, float* absmax, float decay, bool w2d, void* ws, cudaStream_t stream,
-                        void* const* events = nullptr, bool full_ws = true)
+                        void* const* events = nullptr, bool full_ws = true, const NvSource* nv = nullptr)
 {
     // events[0] before the first launch, events[i] after the i-th (measurement hook)
     auto mark = [&](int i) -> bool {
@@ -236,14 +246,22 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         rp.do_row = do_row;
         rp.strided = G == 1;
         rp.x = static_cast<const uint16_t*>(x);
-        rp.amax_row = do_row ? amax_row : nullptr;
+        if (nv) {
+            rp.nq = nv->q;
+            rp.nsf = nv->sf;
+            rp.namax = nv->amax;
+            rp.dscale = nv->dscale;
+            rp.do_row = 0;
+        }
+        rp.amax_row = (do_row && !nv) ? amax_row : nullptr;
         rp.q_row = q_row;
         rp.sf_row = sf_row;
         rp.amax_col = (do_col && !colmax) ? amax_col : nullptr;
         rp.colmax = reinterpret_cast<uint32_t*>(colmax);
         rp.obs = absmax ? ws_obs(ws) : nullptr;
         for (int g = 0; g <= G; ++g) rp.row_off[g] = (int32_t)off[g];
-        if ((e = launch_rowpass<MAXG>(rs, rp, stream)) != cudaSuccess || !mark(2)) return NVFP4PT_ERR_CUDA;
+        e = nv ? launch_rowpass<MAXG, true>(rs, rp, stream) : launch_rowpass<MAXG, false>(rs, rp, stream);
+        if (e != cudaSuccess || !mark(2)) return NVFP4PT_ERR_CUDA;
 
         // Column pass: 256-row tasks per group (the last one ragged) x 32-column strips.
         // With nothing to encode it runs the running-buffer update alone (one CTA).
@@ -271,13 +289,19 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         cp.back_rt = (int32_t)(wstride / cp.strips);
         cp.back_strip = (int32_t)(wstride % cp.strips);
         cp.x = static_cast<const uint16_t*>(x);
+        if (nv) {
+            cp.nq = nv->q;
+            cp.nsf = nv->sf;
+            cp.dscale = nv->dscale;
+        }
         cp.amax_col = amax_col;
         cp.colmax = colmax;
         cp.q_col = q_col;
         cp.sf_col = sf_col;
         cp.absmax = absmax;
         cp.obs = ws_obs(ws);
-        e = launch(colpass<MAXG>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
+        e = nv ? launch(colpass<MAXG, true>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads)
+               : launch(colpass<MAXG, false>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
         return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
     }
 
@@ -328,7 +352,13 @@ cudaError_t launch_dequant(const uint8_t* q, const uint8_t* sf, const float* ama
     return cudaGetLastError();
 }
 
-int64_t requant_bf16_bytes(int64_t rows, int64_t cols) { return align256(rows * cols * 2); }
+// Requantization scratch ahead of the cast's workspace: the rows' decode scales when the
+// row pass can take the NVFP4 data directly (cols <= kRowPassMaxCols), else the whole
+// dequantized matrix (bf16) for the tile path.
+int64_t requant_scratch_bytes(int64_t rows, int64_t cols)
+{
+    return cols <= kRowPassMaxCols ? align256(rows * 4) : align256(rows * cols * 2);
+}
 
 }  // namespace
 
@@ -487,7 +517,7 @@ nvfp4pt_status nvfp4pt_dequantize(const uint8_t* q, const uint8_t* sf, const flo
 size_t nvfp4pt_requantize_workspace_bytes(int64_t rows, int64_t cols, int num_groups)
 {
     const int64_t r = rows < 0 ? 0 : rows, c = cols < 0 ? 0 : cols;
-    return (size_t)requant_bf16_bytes(r, c) + nvfp4pt_workspace_bytes(rows, cols, num_groups);
+    return (size_t)requant_scratch_bytes(r, c) + nvfp4pt_workspace_bytes(rows, cols, num_groups);
 }
 
 nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, const uint8_t* sf_row, const float* amax_row,
@@ -509,9 +539,18 @@ nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, const uint8_t* s
         if (off[g + 1] < off[g] || off[g] % 16) return NVFP4PT_ERR_GROUPS;
     DeviceState* dev = nullptr;
     if ((st = device_state(&dev)) != NVFP4PT_OK) return st;
+    void* ws = static_cast<uint8_t*>(workspace) + requant_scratch_bytes(rows, cols);
+    if (cols <= kRowPassMaxCols) {
+        // the row pass and the column pass read the NVFP4 data themselves
+        const NvSource src{q_row, sf_row, amax_row, static_cast<float*>(workspace)};
+        if (G == 1)
+            return run_cast<1>(nullptr, rows, cols, off, 1, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col,
+                               sf_col, amax_col, absmax_bufs, decay, false, ws, stream, nullptr, true, &src);
+        return run_cast<kMaxGroups>(nullptr, rows, cols, off, G, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col,
+                                    sf_col, amax_col, absmax_bufs, decay, false, ws, stream, nullptr, true, &src);
+    }
     // X' (bf16) in the workspace, then the columnwise cast of X' with the rest of it
     uint16_t* xd = static_cast<uint16_t*>(workspace);
-    void* ws = static_cast<uint8_t*>(workspace) + requant_bf16_bytes(rows, cols);
     if (launch_dequant(q_row, sf_row, amax_row, rows, cols, xd, dev->sm_count, stream) != cudaSuccess)
         return NVFP4PT_ERR_CUDA;
     if (G == 1)

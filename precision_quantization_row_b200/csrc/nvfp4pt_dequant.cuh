@@ -52,6 +52,33 @@ __device__ __forceinline__ uint32_t scale_to_bf16x2(float t0, float t1, float m)
     return r;
 }
 
+// Dequantized values of four consecutive elements (codes4: 4 nibbles, element 0 in the
+// low nibble) with block scale s (the decoded E4M3 value) and decode scale m, as two
+// bf16x2 words (elements 0,1 and 2,3; first element in the low half).
+__device__ __forceinline__ void dequant4(uint32_t codes4, float s, float m, uint32_t& w01, uint32_t& w23)
+{
+    uint32_t b01, b23;
+    e2m1x4_to_bf16(codes4, b01, b23);
+    float t0, t1, t2, t3;
+    mul2(t0, t1, bf16_lo(b01), bf16_hi(b01), s);   // val * float(sf): exact
+    mul2(t2, t3, bf16_lo(b23), bf16_hi(b23), s);
+    w01 = scale_to_bf16x2(t0, t1, m);
+    w23 = scale_to_bf16x2(t2, t3, m);
+}
+
+// One 16-element block (8 code bytes c8, scale code sfc, decode scale m) as the eight
+// bf16x2 words a 32-byte load of the same block of x would give.
+__device__ __forceinline__ void dequant16(uint2 c8, uint32_t sfc, float m, uint32_t (&w)[8])
+{
+    float s, s_unused;
+    e4m3x2_decode(sfc & 0xFFu, s, s_unused);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t word = (h < 2) ? c8.x : c8.y;
+        dequant4((word >> (16 * (h & 1))) & 0xFFFFu, s, m, w[2 * h], w[2 * h + 1]);
+    }
+}
+
 __global__ void __launch_bounds__(256) dequant_rows_kernel(const __grid_constant__ DequantParams p)
 {
     const int64_t bpr = p.cols / 16;   // blocks per row
@@ -60,23 +87,8 @@ __global__ void __launch_bounds__(256) dequant_rows_kernel(const __grid_constant
         for (int64_t j = threadIdx.x; j < bpr; j += blockDim.x) {
             const int64_t b = row * bpr + j;
             const uint2 c8 = *reinterpret_cast<const uint2*>(p.q + 8 * b);   // 16 codes, element 2i low nibble
-            float s, s_unused;
-            e4m3x2_decode(p.sf[b], s, s_unused);
             uint32_t out[8];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                // codes of elements 4h..4h+3: byte pair h of the 8 code bytes
-                const uint32_t w = (h < 2) ? c8.x : c8.y;
-                const uint32_t codes4 = (w >> (16 * (h & 1))) & 0xFFFFu;
-                uint32_t b01, b23;
-                e2m1x4_to_bf16(codes4, b01, b23);
-                // val * float(sf): exact, from the bf16 magnitudes
-                float t0, t1, t2, t3;
-                mul2(t0, t1, bf16_lo(b01), bf16_hi(b01), s);
-                mul2(t2, t3, bf16_lo(b23), bf16_hi(b23), s);
-                out[2 * h] = scale_to_bf16x2(t0, t1, m);
-                out[2 * h + 1] = scale_to_bf16x2(t2, t3, m);
-            }
+            dequant16(c8, p.sf[b], m, out);
             uint4* dst = reinterpret_cast<uint4*>(p.out + 16 * b);
             dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
             dst[1] = make_uint4(out[4], out[5], out[6], out[7]);

@@ -433,6 +433,14 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p)
     return v;
 }
 
+// 8 bytes through the read-only path, not kept in L1.
+__device__ __forceinline__ uint2 ldg_stream64(const void* p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
 // 32 bytes (one 16-element bf16 block) through the read-only path, not kept in L1.
 __device__ __forceinline__ void ldg256_stream(const void* p, uint32_t (&v)[8])
 {
