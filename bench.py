@@ -421,6 +421,90 @@ def run_gpu_op(args, dist: Dist, op: str) -> dict | None:
     }
 
 
+def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
+    """Device time per call of the other workloads (parity-test configurations, reported
+    beside the headline): dense 4096x4096 row+column cast, the grouped MoE cast
+    (65536x7168, 64 token groups) and the 16x16 weight cast (28672x8192). Two input
+    copies rotate (the dense one fits L2: 8 copies rotate there)."""
+    import torch
+
+    import precision_quantization_row_b200 as nv
+    from precision_quantization_row_b200 import build, inputs
+
+    build.build()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    stream = torch.cuda.current_stream(dev)
+    if config == "dense":
+        x = inputs.dense().to(dev)
+        m, k, g, copies = x.shape[0], x.shape[1], 1, 8
+    elif config == "moe":
+        xh, offsets = inputs.moe()
+        x = xh.to(dev)
+        m, k, g, copies = x.shape[0], x.shape[1], len(offsets) - 1, 2
+    else:
+        x = inputs.weight().to(dev)
+        m, k, g, copies = x.shape[0], x.shape[1], 1, 2
+    xs = [x] + [x.clone() for _ in range(copies - 1)]
+    ws = nv.new_workspace(m, k, g, device=dev)
+    if config == "moe":
+        outs = [None] * copies
+        bufs = torch.zeros(g, dtype=torch.float32, device=dev)
+
+        def step(i):
+            outs[i % copies] = nv.quantize_grouped(xs[i % copies], offsets, absmax=bufs, decay=DECAY,
+                                                   out=outs[i % copies], workspace=ws, stream=stream)
+        byts = 2 * (2 * m * k) + 2 * (m * k // 2) + 2 * (m * k // 16) + 4 * m + 4 * g * k
+    elif config == "dense":
+        outs = [nv._outputs(m, k, nv.ROWWISE | nv.COLWISE, dev) for _ in range(copies)]
+        buf = torch.zeros(1, dtype=torch.float32, device=dev)
+
+        def step(i):
+            nv.quantize(xs[i % copies], absmax=buf, decay=DECAY, out=outs[i % copies], workspace=ws, stream=stream)
+        byts = algo_bytes(m, k)
+    else:
+        outs = [None] * copies
+
+        def step(i):
+            outs[i % copies] = nv.quantize_weight_2d(xs[i % copies], out=outs[i % copies], workspace=ws,
+                                                     stream=stream)
+        byts = 2 * (2 * m * k) + m * k // 2 + m * k // 16 + 4 * m   # read twice, rowwise out
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run():
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1) / 1e3
+
+    with ClockSampler(dev.index) as clk:
+        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    if nv.workspace_error(ws) != 0:
+        raise RuntimeError("device error word set during the timed region")
+    if dist.rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    per = secs / args.steps
+    achieved = byts / per / 1e9
+    return {
+        "metric": "NVFP4 per-token cast: elems/s, achieved HBM GB/s, % of B200 HBM peak",
+        "value": float(m) * k * args.steps * dist.world / secs, "unit": "elem/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16->nvfp4", "data": "synthetic",
+        "config": {"workload": {"dense": "dense_4096x4096_rowcol", "moe": "moe_grouped_65536x7168_g64_rowcol",
+                                "weight": "weight_2d_28672x8192"}[config],
+                   "rows": m, "cols": k, "groups": g, "l2": f"{copies} rotating input copies"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_kind, "algorithmic_bytes_per_call": byts},
+        "clocks": clk.summary(),
+    }
+
+
 def oracle_sample_rate(rows: int) -> tuple[float, str]:
     """elems/s of the oracle's full row+col cast (with the absmax update) of the
     first `rows` rows of the benchmark matrix, single-threaded."""
@@ -483,6 +567,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--op", choices=["cast", "dequant", "requant"], default="cast",
                     help="cast: the per-token cast (the headline); dequant / requant: the secondary ops")
+    ap.add_argument("--config", choices=["llm", "dense", "moe", "weight"], default="llm",
+                    help="llm: the headline activation; the others time the remaining workloads")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -492,6 +578,14 @@ def main(argv=None):
             print(json.dumps(line), flush=True)
         return
     dist = Dist(args.gpus)
+    if args.config != "llm":
+        try:
+            line = run_gpu_config(args, dist, args.config)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+        finally:
+            dist.close()
+        return
     if args.op != "cast":
         try:
             line = run_gpu_op(args, dist, args.op)
