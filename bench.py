@@ -21,6 +21,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -62,11 +63,24 @@ def kernel_bytes(name: str, m: int, k: int) -> int:
     return 4 * k
 
 
-def kernel_source_sha() -> str:
+def strip_comments(src: str) -> str:
+    """C/C++ source without comments and blank space, so that the hash below changes
+    with the code only (string literals here hold no comment markers)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def kernel_source_sha(texts=None) -> str:
+    """Hash of the kernel sources' code (comments and spacing do not count)."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+    if texts is None:
+        texts = []
+        for p in KERNEL_SOURCES:
+            with open(p, encoding="utf-8") as f:
+                texts.append(f.read())
+    for t in texts:
+        h.update(strip_comments(t).encode())
     return h.hexdigest()[:16]
 
 

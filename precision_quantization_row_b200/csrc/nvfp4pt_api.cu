@@ -1,6 +1,8 @@
-// Host side of the C ABI declared in include/nvfp4pt.h: argument checks, the TMA
-// descriptor of x, and the launches (zero -> amax pass -> encode pass, chained with
-// programmatic dependent launch on the caller's stream).
+// Host side of the C ABI declared in include/nvfp4pt.h and nvfp4pt_timing.h: argument
+// checks, the workspace layout, and the launches on the caller's stream (zero -> amax
+// pass -> encode pass, chained with programmatic dependent launch): the row pass and
+// the column pass for rows up to 16384 elements (also from NVFP4 rowwise data, for the
+// requantization), else the TMA tile path; the dequantization kernel.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

@@ -24,7 +24,7 @@ constexpr uint32_t kWaitLimit = 1u << 22;     // try_wait rounds before giving u
 
 // ------------------------------------------------------------------ geometry
 //
-// Both passes walk the same sequence of 128 x 128 tiles: for each token group g
+// Both passes of the tile path walk the same sequence of 128 x 128 tiles: for each token group g
 // (one group when ungrouped), its rows split into 128-row bands (the last band of a
 // group may be shorter, a multiple of 16), each band into ceil(cols/128) column
 // tiles. Tile t is band t / ntc, column tile t % ntc. CTA c of both passes owns the

@@ -1,7 +1,10 @@
-// Kernels of the NVFP4 per-token cast (sm_100a).
+// Kernels of the NVFP4 per-token cast (sm_100a) shared by every route, and the tile
+// path (the 16x16 weight cast and rows wider than 16384 elements; the 1D casts of
+// narrower rows run the row pass and the column pass of nvfp4pt_rowpass.cuh and
+// nvfp4pt_colpass.cuh instead).
 //
-//   pass0_zero   zeroes the amax outputs and the per-call scratch (the maxima below
-//                are accumulated with atomic max on non-negative float bits).
+//   pass0_zero   zeroes the amax outputs and the per-call scratch (the maxima are
+//                accumulated with atomic max on non-negative float or bf16 bits).
 //   pass1_amax   the vector-amax stage of TransformerEngine PR #3045 (its "K1"): one
 //                read of x gives the per-row amax, the per-column amax (per token
 //                group when grouped) and the observed maximum of the running buffer.
