@@ -49,8 +49,9 @@ def _rows_of(x):
     return out["q_row"], out["sf_row"], out["amax_row"]
 
 
-# (64, 16400): rows wider than 16384 take the dequantize-then-cast route
-@pytest.mark.parametrize("shape", [(256, 512), (1040, 1056), (4096, 4096), (48, 80), (64, 16400)],
+# (64, 12288): two blocks per row-pass thread; (64, 16400): rows wider than 16384 take
+# the dequantize-then-cast route
+@pytest.mark.parametrize("shape", [(256, 512), (1040, 1056), (4096, 4096), (48, 80), (64, 12288), (64, 16400)],
                          ids=lambda s: f"{s[0]}x{s[1]}")
 def test_requant_colwise(orc, shape):
     x = inputs.random_shape(62, *shape, "wide")
