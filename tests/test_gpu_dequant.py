@@ -76,6 +76,16 @@ def test_requant_grouped(orc):
     assert np.array_equal(bufs.cpu().numpy().view(np.uint32), want["absmax"].view(np.uint32))
 
 
+def test_requant_grouped_wide_rows(orc):
+    """Grouped requantization of rows 12288 wide (two blocks per row-pass thread)."""
+    x = inputs.random_shape(65, 128, 12288, "normal")
+    offsets = [0, 64, 64, 128]
+    q, sf, a = _rows_of(x)
+    got = nv.requantize_colwise(q, sf, a, offsets=offsets)
+    want = orc.requantize_colwise(q.cpu().numpy(), sf.cpu().numpy(), a.cpu().numpy(), offsets=offsets)
+    compare(to_np(got), {k: want[k] for k in ("q_col", "sf_col", "amax_col")}, label="grouped requant wide")
+
+
 def test_requant_of_lossless_rows_equals_direct_cast():
     """Rows whose cast is lossless: requantizing their rowwise data on the GPU gives the
     GPU's direct columnwise cast of the matrix itself."""

@@ -218,6 +218,20 @@ def test_grouped(orc, rows, offsets):
     compare(got, want, label=f"grouped {offsets}")
 
 
+@pytest.mark.parametrize("cols", [12288, 16400], ids=["two_blocks_per_thread", "tile_path"])
+def test_grouped_wide_rows(orc, cols):
+    """Grouped cast of rows 8192..16384 wide (two blocks per row-pass thread) and wider
+    than 16384 (the tile path), with an empty group and a ragged one."""
+    offsets = [0, 48, 48, 112, 128]
+    x = inputs.random_shape(cols, 128, cols, "wide")
+    G = len(offsets) - 1
+    bufs = torch.full((G,), 1.0, dtype=torch.float32, device="cuda")
+    got = to_np(nv.quantize_grouped(x.cuda(), offsets, absmax=bufs, decay=0.25))
+    want = orc.quantize_grouped(x, offsets, absmax=np.full(G, 1.0, np.float32), decay=0.25)
+    got["absmax"] = bufs.cpu().numpy()
+    compare(got, want, label=f"grouped wide {cols}")
+
+
 def test_grouped_many_groups(orc):
     rng = np.random.default_rng(15)
     G = 1024
