@@ -349,8 +349,14 @@ cudaError_t launch_dequant(const uint8_t* q, const uint8_t* sf, const float* ama
     d.out = out;
     d.rows = rows;
     d.cols = cols;
-    const int grid = (int)std::min<int64_t>(rows, 8 * (int64_t)sm_count);
-    dequant_rows_kernel<<<grid, 256, 0, stream>>>(d);
+    d.out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+    // two blocks per thread when rows hold an even number of blocks (a pair never spans
+    // two rows); the grid covers every unit once, up to 128 CTAs per SM
+    const bool pairs = (cols / 16) % 2 == 0;
+    d.units = rows * (cols / 16) / (pairs ? 2 : 1);
+    const int grid = (int)std::min<int64_t>((d.units + 255) / 256, 128 * (int64_t)sm_count);
+    if (pairs) dequant_rows_kernel<2><<<grid, 256, 0, stream>>>(d);
+    else dequant_rows_kernel<1><<<grid, 256, 0, stream>>>(d);
     return cudaGetLastError();
 }
 

@@ -5,9 +5,11 @@
 // the TransformerEngine pages store beside the block scales). val(q) * float(sf) is
 // exact in binary32. Columnwise data ([cols, rows/2], ...) give X^T the same way.
 //
-// CTAs take rows (grid-strided), threads the 16-element blocks of a row: 8 code bytes
-// and one scale byte in, 32 bytes out; the row's decode scale once per row and
-// thread. HBM-bound: 0.5625 B read and 2 B written per element.
+// Each thread takes one unit of one or two blocks of a row (two when a row holds an even
+// number of blocks): 8 or 16 code bytes and the units' scale bytes in, 32 bytes out per
+// block, the row's decode scale recomputed per unit. The grid covers every unit once
+// up to 128 CTAs per SM and strides beyond that; the short life of each thread keeps
+// loads of many units in flight. HBM-bound: 0.5625 B read and 2 B written per element.
 #pragma once
 
 #include "nvfp4pt_device.cuh"
@@ -21,6 +23,8 @@ struct DequantParams {
     uint16_t* out;
     int64_t rows;
     int64_t cols;
+    int64_t units;    // rows * cols / (16 * blocks per unit)
+    int32_t out32;    // out is 32-byte aligned: one store per block
 };
 
 // The E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 are bf16 values: high bytes
@@ -79,19 +83,39 @@ __device__ __forceinline__ void dequant16(uint2 c8, uint32_t sfc, float m, uint3
     }
 }
 
-__global__ void __launch_bounds__(256) dequant_rows_kernel(const __grid_constant__ DequantParams p)
+// The 32 output bytes of one block.
+__device__ __forceinline__ void store_block(uint16_t* dst, const uint32_t (&w)[8], bool out32)
 {
-    const int64_t bpr = p.cols / 16;   // blocks per row
-    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
-        const float m = __fdiv_rn(p.amax[row], 2688.0f);   // decode scale of the row
-        for (int64_t j = threadIdx.x; j < bpr; j += blockDim.x) {
-            const int64_t b = row * bpr + j;
-            const uint2 c8 = *reinterpret_cast<const uint2*>(p.q + 8 * b);   // 16 codes, element 2i low nibble
-            uint32_t out[8];
-            dequant16(c8, p.sf[b], m, out);
-            uint4* dst = reinterpret_cast<uint4*>(p.out + 16 * b);
-            dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-            dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    uint8_t* d = reinterpret_cast<uint8_t*>(dst);
+    if (out32) {
+        stg32(d, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+    } else {
+        *reinterpret_cast<uint4*>(d) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(d + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
+// BPT blocks (1 or 2) per unit; units are numbered row-major, so unit u starts at
+// block BPT * u of the flat [rows, cols / 16] block grid.
+template <int BPT>
+__global__ void __launch_bounds__(256, 8) dequant_rows_kernel(const __grid_constant__ DequantParams p)
+{
+    const int64_t upr = p.cols / (16 * BPT);   // units per row
+    const int64_t stride = (int64_t)gridDim.x * 256;
+    for (int64_t u = (int64_t)blockIdx.x * 256 + threadIdx.x; u < p.units; u += stride) {
+        const float m = __fdiv_rn(__ldg(p.amax + u / upr), 2688.0f);   // decode scale of the row
+        uint32_t w[8];
+        if constexpr (BPT == 2) {
+            const uint4 c = __ldg(reinterpret_cast<const uint4*>(p.q + 16 * u));   // element 2i low nibble
+            const uint32_t s = __ldg(reinterpret_cast<const uint16_t*>(p.sf) + u);
+            dequant16(make_uint2(c.x, c.y), s & 0xFFu, m, w);
+            store_block(p.out + 32 * u, w, p.out32);
+            dequant16(make_uint2(c.z, c.w), s >> 8, m, w);
+            store_block(p.out + 32 * u + 16, w, p.out32);
+        } else {
+            const uint2 c = __ldg(reinterpret_cast<const uint2*>(p.q + 8 * u));
+            dequant16(c, __ldg(p.sf + u), m, w);
+            store_block(p.out + 16 * u, w, p.out32);
         }
     }
 }

@@ -35,6 +35,32 @@ def test_dequant_random_codes(orc, shape):
     assert bad.size == 0, f"{bad.shape[0]} mismatches, first {bad[:3].tolist()}"
 
 
+@pytest.mark.parametrize("shape", [(272, 1056), (48, 80)], ids=lambda s: f"{s[0]}x{s[1]}")
+def test_dequant_output_16_byte_aligned(orc, shape):
+    """An output 16 bytes past a 32-byte boundary: each block goes out as two 16-byte
+    stores (rows with an even and an odd number of blocks)."""
+    q, sf, amax = _random_rows(70, *shape)
+    rows, cols = shape
+    buf = torch.empty(rows * cols + 8, dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(rows, cols)
+    assert out.data_ptr() % 32 == 16
+    nv.dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), torch.from_numpy(amax).cuda(), out=out)
+    want = orc.dequantize(q, sf, amax)
+    assert np.array_equal(out.cpu().view(torch.int16).numpy().view(np.uint16), want)
+
+
+# more units (two blocks each, then one block each for rows of 1025 blocks) than the
+# grid's threads at 128 CTAs per SM: threads take several units
+@pytest.mark.parametrize("shape", [(10240, 16384), (6144, 16400)], ids=lambda s: f"{s[0]}x{s[1]}")
+def test_dequant_grid_stride(orc, shape):
+    q, sf, amax = _random_rows(sum(shape), *shape)
+    got = nv.dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), torch.from_numpy(amax).cuda())
+    want = orc.dequantize(q, sf, amax)
+    g = got.cpu().view(torch.int16).numpy().view(np.uint16)
+    bad = np.argwhere(g != want)
+    assert bad.size == 0, f"{bad.shape[0]} mismatches, first {bad[:3].tolist()}"
+
+
 @pytest.mark.parametrize("kind", ["normal", "wide", "tiny", "signed_zero"])
 def test_dequant_of_cast_outputs(orc, kind):
     x = inputs.random_shape(61, 512, 768, kind).cuda()
