@@ -119,8 +119,7 @@ template <typename Kernel, typename Params>
 cudaError_t launch(Kernel kernel, int grid, int smem, cudaStream_t stream, const Params& p, bool pdl,
                    int threads = kThreads)
 {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof cfg);
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = (size_t)smem;

@@ -205,12 +205,6 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
     return r;
 }
 
-// Four zero-extended bytes -> one word, b0 in bits 0-7.
-__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3)
-{
-    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-}
-
 // (y0, y1) = (RN(x0 * e), RN(x1 * e)) with one packed two-lane binary32 multiply.
 __device__ __forceinline__ void mul2(float& y0, float& y1, float x0, float x1, float e)
 {
@@ -219,14 +213,6 @@ __device__ __forceinline__ void mul2(float& y0, float& y1, float x0, float x1, f
     asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(e));
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(d));
-}
-
-// Codes of the pair (x0, x1) scaled by e: one byte, x0 in the low nibble.
-__device__ __forceinline__ uint32_t code_pair(float x0, float x1, float e)
-{
-    float y0, y1;
-    mul2(y0, y1, x0, x1, e);
-    return e2m1x2(y0, y1);
 }
 
 // Two E4M3 (e4m3fn) codes, round-to-nearest-even, saturating: `lo` -> bits 0-7,
