@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_f32_to_bf16_array.argtypes, _lib.oracle_f32_to_bf16_array.restype = [P, I64, P], None
         _lib.oracle_dequantize_rows.argtypes = [P, P, P, I64, I64, P]
         _lib.oracle_dequantize_rows.restype = ctypes.c_int
+        _lib.oracle_gemm_per_token.argtypes = [P, P, P, I64, P, P, P, I64, I64, P, P]
+        _lib.oracle_gemm_per_token.restype = ctypes.c_int
     return _lib
 
 
@@ -285,3 +287,30 @@ def requantize_colwise(q_row, sf_row, amax_row, offsets=None, absmax=None, decay
     if "absmax" in out:
         res["absmax"] = out["absmax"]
     return res
+
+
+def gemm_per_token(qa, sfa, amax_a, qb, sfb, amax_b):
+    """oracle_gemm_per_token: D [M, N] (float64) of two K-major rowwise-layout NVFP4
+    operands (A: q [M, K/2], sf [M, K/16], amax [M]; B: q [N, K/2], sf [N, K/16],
+    amax [N]), D = S_dec(amax_a) S_dec(amax_b) * sum_k val*sf*val*sf with the sum
+    exact; also the same expression over the terms' magnitudes, [M, N]."""
+    qa = np.ascontiguousarray(np.asarray(qa, np.uint8))
+    qb = np.ascontiguousarray(np.asarray(qb, np.uint8))
+    M, half = qa.shape
+    N = qb.shape[0]
+    K = 2 * half
+    if qb.shape[1] != half:
+        raise ValueError("operands differ in K")
+    sa = np.ascontiguousarray(np.asarray(sfa, np.uint8).reshape(M, K // 16))
+    sb = np.ascontiguousarray(np.asarray(sfb, np.uint8).reshape(N, K // 16))
+    aa = np.ascontiguousarray(np.asarray(amax_a, np.float32).reshape(M))
+    ab = np.ascontiguousarray(np.asarray(amax_b, np.float32).reshape(N))
+    out = np.zeros((M, N), np.float64)
+    mag = np.zeros((M, N), np.float64)
+    st = lib().oracle_gemm_per_token(_ptr(qa), _ptr(sa), _ptr(aa), M, _ptr(qb), _ptr(sb), _ptr(ab), N, K,
+                                     _ptr(out), _ptr(mag))
+    if st == -1:
+        raise ValueError(f"oracle_gemm_per_token: bad shape M={M} N={N} K={K}")
+    if st == -2:
+        raise ValueError("oracle_gemm_per_token: a block scale is not a non-negative finite e4m3fn code")
+    return out, mag

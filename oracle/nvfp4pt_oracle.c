@@ -29,6 +29,9 @@
  *    per-token scaling the observed value is the row amaxes max-reduced to a scalar.
  *  - TransformerEngine PR #3244 (row-wise pre-quantized grouped GEMM input),
  *    review: "compact" scales means the unswizzled row-major layout.
+ *  - TransformerEngine PR #3045, Changes and Greptile summary: the per-token GEMM
+ *    over NVFP4 operands, rescaled by the per-row and per-column outer-amax
+ *    vectors in its epilogue (oracle_gemm_per_token, with its reading).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - s_enc = 1 when amax == 0; an overflowing 2688/amax (amax below ~7.9e-36)
@@ -392,6 +395,71 @@ int oracle_dequantize_rows(const uint8_t* q, const uint8_t* sf, const float* ama
                 const float y = t * sdec;
                 out[r * K + 16 * b + j] = oracle_f32_to_bf16(y);
             }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------- per-token GEMM */
+
+/* 2 * val(code) for an E2M1 code (integer: -12..12; -0 gives 0). */
+static int64_t e2m1_twice(uint8_t code)
+{
+    static const int64_t kTwice[8] = {0, 1, 2, 3, 4, 6, 8, 12};
+    const int64_t v = kTwice[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+/* 2^9 * float(sf) for a non-negative finite e4m3fn code 0..126 (an integer:
+ * subnormals are m * 2^-9, normals (8 + m) * 2^(e - 10) with e >= 1); -1 for any
+ * other code. */
+static int64_t e4m3_times_512(uint8_t code)
+{
+    if (code > 0x7E) return -1;
+    return (int64_t)ldexp(e4m3_magnitude(code), 9);
+}
+
+/* The per-token NVFP4 GEMM (TransformerEngine PR #3045, Changes and the Greptile
+ * summary: a GEMM over the per-token NVFP4 operands that applies the per-row and
+ * per-column outer-amax vectors in its epilogue; the call takes each operand's
+ * codes, block scales and amax vector and returns an M x N output). The reading
+ * taken: both operands are K-major rowwise-layout NVFP4 data,
+ *     A: codes [M, K/2], scales [M, K/16], amax [M];  B: [N, K/2], [N, K/16], [N],
+ * and, with S_dec(a) = RN(a / 2688) the binary32 decode scale of the dequantization,
+ *     D[m][n] = S_dec(amax_a[m]) * S_dec(amax_b[n])
+ *               * sum_k val(qa[m][k]) sf_a[m][k/16] val(qb[n][k]) sf_b[n][k/16].
+ * Every term is a whole multiple of 2^-20 (val is a multiple of 1/2, sf of 2^-9),
+ * so the sum is taken exactly in integers in units of 2^-20 and rounded once to
+ * double; the product of the two decode scales (exact in double) then multiplies
+ * it with one more rounding, the same for D(A, B) and D(B, A)^T. abs_out (optional) gets
+ * the same expression over the terms' magnitudes: the scale of the rounding error
+ * of any binary32 evaluation. Returns -1 for a bad shape, -2 for a scale code that
+ * is not a non-negative finite e4m3fn value. */
+int oracle_gemm_per_token(const uint8_t* qa, const uint8_t* sfa, const float* amax_a, int64_t M,
+                          const uint8_t* qb, const uint8_t* sfb, const float* amax_b, int64_t N,
+                          int64_t K, double* out, double* abs_out)
+{
+    if (M < 1 || N < 1 || K < 16 || K % 16) return -1;
+    for (int64_t i = 0; i < M * (K / 16); ++i)
+        if (e4m3_times_512(sfa[i]) < 0) return -2;
+    for (int64_t i = 0; i < N * (K / 16); ++i)
+        if (e4m3_times_512(sfb[i]) < 0) return -2;
+    for (int64_t m = 0; m < M; ++m) {
+        const double sa = (double)(amax_a[m] / 2688.0f);
+        for (int64_t n = 0; n < N; ++n) {
+            const double scale = sa * (double)(amax_b[n] / 2688.0f);   /* exact: 24 + 24 bits */
+            __int128 acc = 0, acc_abs = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                const uint8_t ba = qa[m * (K / 2) + k / 2], bb = qb[n * (K / 2) + k / 2];
+                const uint8_t ca = (k & 1) ? (uint8_t)(ba >> 4) : (uint8_t)(ba & 0xF);
+                const uint8_t cb = (k & 1) ? (uint8_t)(bb >> 4) : (uint8_t)(bb & 0xF);
+                const int64_t t = e2m1_twice(ca) * e2m1_twice(cb) * e4m3_times_512(sfa[m * (K / 16) + k / 16]) *
+                                  e4m3_times_512(sfb[n * (K / 16) + k / 16]);   /* |t| < 2^43 */
+                acc += t;
+                acc_abs += t < 0 ? -t : t;
+            }
+            out[m * N + n] = ldexp((double)acc, -20) * scale;
+            if (abs_out) abs_out[m * N + n] = ldexp((double)acc_abs, -20) * fabs(scale);
         }
     }
     return 0;
