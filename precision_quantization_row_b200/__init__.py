@@ -13,6 +13,7 @@ Names follow the C entry points (nvfp4pt_quantize -> quantize, ...).
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -89,7 +90,7 @@ def _check(fn: str, status: int) -> None:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream, device):
@@ -97,13 +98,60 @@ def _stream(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _require_cuda_bf16(x: torch.Tensor, name: str):
-    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+def _require_2d(x, name: str, dtype) -> None:
+    if not isinstance(x, torch.Tensor) or x.dtype != dtype or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous 2D {dtype} tensor")
+
+
+def _require_cuda(x: torch.Tensor, name: str) -> None:
+    if not x.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor (there is no CPU path)")
-    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
-        raise TypeError(f"{name} must be a contiguous 2D bfloat16 tensor")
 
 
+# The C ABI takes raw pointers and cannot see buffer sizes, so the binding checks what
+# the kernels rely on before any call: each buffer's dtype, contiguity, element count
+# and device (that of the call's main input; CPU tensors meet the same checks, and the
+# main input's "must be CUDA" check comes last).
+def _buf(t, name: str, dtype, n: int, dev: int) -> int:
+    try:
+        if t.dtype is dtype and t.numel() >= n and t.is_contiguous() and t.get_device() == dev:
+            return t.data_ptr()
+    except AttributeError:   # not a tensor
+        pass
+    raise _bad_buf(t, name, dtype, n, dev)
+
+
+def _bad_buf(t, name: str, dtype, n: int, dev: int) -> Exception:
+    if not isinstance(t, torch.Tensor):
+        return TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype is not dtype:
+        return TypeError(f"{name} must be {dtype}, not {t.dtype}")
+    if not t.is_contiguous():
+        return ValueError(f"{name} must be contiguous")
+    if t.numel() < n:
+        return ValueError(f"{name} holds {t.numel()} elements, the call needs {n}")
+    return TypeError(f"{name} is on device {t.get_device()}, the call's input on {dev}")
+
+
+def _out_ptrs(out: dict, flags: int, rows: int, cols: int, groups: int, dev: int) -> list:
+    """Pointers of the cast's outputs for `flags` (None for the direction not asked for)."""
+    p = [None] * 6
+    if flags & ROWWISE:
+        p[0] = _buf(out.get("q_row"), "q_row", torch.uint8, rows * cols // 2, dev)
+        p[1] = _buf(out.get("sf_row"), "sf_row", torch.uint8, rows * cols // 16, dev)
+        p[2] = _buf(out.get("amax_row"), "amax_row", torch.float32, rows, dev)
+    if flags & COLWISE:
+        p[3] = _buf(out.get("q_col"), "q_col", torch.uint8, cols * rows // 2, dev)
+        p[4] = _buf(out.get("sf_col"), "sf_col", torch.uint8, cols * rows // 16, dev)
+        p[5] = _buf(out.get("amax_col"), "amax_col", torch.float32, groups * cols, dev)
+    return p
+
+
+def _opt_buf(t, name: str, dtype, n: int, dev: int):
+    return None if t is None else _buf(t, name, dtype, n, dev)
+
+
+@functools.lru_cache(maxsize=256)
 def workspace_bytes(rows: int, cols: int, num_groups: int = 1) -> int:
     return int(lib().nvfp4pt_workspace_bytes(rows, cols, num_groups))
 
@@ -134,14 +182,17 @@ def quantize(x: torch.Tensor, flags: int = ROWWISE | COLWISE, absmax: torch.Tens
              decay: float = 0.0, out: dict | None = None, workspace: torch.Tensor | None = None,
              stream: torch.cuda.Stream | None = None) -> dict:
     """nvfp4pt_quantize. absmax: optional fp32 CUDA tensor of one element, updated in place."""
-    _require_cuda_bf16(x, "x")
+    _require_2d(x, "x", torch.bfloat16)
     rows, cols = x.shape
+    dev = x.get_device()
     out = _outputs(rows, cols, flags, x.device) if out is None else out
     ws = new_workspace(rows, cols, 1, x.device) if workspace is None else workspace
-    st = lib().nvfp4pt_quantize(
-        _ptr(x), rows, cols, flags, _ptr(out.get("q_row")), _ptr(out.get("sf_row")), _ptr(out.get("amax_row")),
-        _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("amax_col")), _ptr(absmax),
-        ctypes.c_float(decay), _ptr(ws), _stream(stream, x.device))
+    p = _out_ptrs(out, flags, rows, cols, 1, dev)
+    pa = _opt_buf(absmax, "absmax", torch.float32, 1, dev)
+    pw = _buf(ws, "workspace", torch.uint8, workspace_bytes(rows, cols, 1), dev)
+    _require_cuda(x, "x")
+    st = lib().nvfp4pt_quantize(_ptr(x), rows, cols, flags, *p, pa, ctypes.c_float(decay), pw,
+                                _stream(stream, x.device))
     _check("nvfp4pt_quantize", st)
     return out
 
@@ -155,17 +206,20 @@ def quantize_timed(x: torch.Tensor, events, flags: int = ROWWISE | COLWISE, absm
     """nvfp4pt_quantize_timed: quantize with events[0] recorded before the first kernel
     launch and events[i] after the i-th (CAST_LAUNCHES + 1 torch.cuda.Event objects,
     created with enable_timing=True and already recorded once, so that they exist)."""
-    _require_cuda_bf16(x, "x")
+    _require_2d(x, "x", torch.bfloat16)
     if len(events) != CAST_LAUNCHES + 1:
         raise ValueError(f"need {CAST_LAUNCHES + 1} events")
     rows, cols = x.shape
+    dev = x.get_device()
     out = _outputs(rows, cols, flags, x.device) if out is None else out
     ws = new_workspace(rows, cols, 1, x.device) if workspace is None else workspace
+    p = _out_ptrs(out, flags, rows, cols, 1, dev)
+    pa = _opt_buf(absmax, "absmax", torch.float32, 1, dev)
+    pw = _buf(ws, "workspace", torch.uint8, workspace_bytes(rows, cols, 1), dev)
+    _require_cuda(x, "x")
     evs = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
-    st = lib().nvfp4pt_quantize_timed(
-        _ptr(x), rows, cols, flags, _ptr(out.get("q_row")), _ptr(out.get("sf_row")), _ptr(out.get("amax_row")),
-        _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("amax_col")), _ptr(absmax),
-        ctypes.c_float(decay), _ptr(ws), _stream(stream, x.device), evs)
+    st = lib().nvfp4pt_quantize_timed(_ptr(x), rows, cols, flags, *p, pa, ctypes.c_float(decay), pw,
+                                      _stream(stream, x.device), evs)
     _check("nvfp4pt_quantize_timed", st)
     return out
 
@@ -174,17 +228,21 @@ def dequantize(q: torch.Tensor, sf: torch.Tensor, amax: torch.Tensor, out: torch
                stream: torch.cuda.Stream | None = None) -> torch.Tensor:
     """nvfp4pt_dequantize: rowwise-layout NVFP4 data (q uint8 [rows, cols/2], sf uint8
     [rows, cols/16], amax fp32 [rows]) back to bf16 [rows, cols]."""
-    for t, n in ((q, "q"), (sf, "sf"), (amax, "amax")):
-        if not t.is_cuda:
-            raise ValueError(f"{n} must be a CUDA tensor")
+    _require_2d(q, "q", torch.uint8)
     rows, half = q.shape
     cols = 2 * half
+    dev = q.get_device()
+    ps = _buf(sf, "sf", torch.uint8, rows * cols // 16, dev)
+    pa = _buf(amax, "amax", torch.float32, rows, dev)
     out = torch.empty((rows, cols), dtype=torch.bfloat16, device=q.device) if out is None else out
-    st = lib().nvfp4pt_dequantize(_ptr(q), _ptr(sf), _ptr(amax), rows, cols, _ptr(out), _stream(stream, q.device))
+    po = _buf(out, "out", torch.bfloat16, rows * cols, dev)
+    _require_cuda(q, "q")
+    st = lib().nvfp4pt_dequantize(_ptr(q), ps, pa, rows, cols, po, _stream(stream, q.device))
     _check("nvfp4pt_dequantize", st)
     return out
 
 
+@functools.lru_cache(maxsize=256)
 def requantize_workspace_bytes(rows: int, cols: int, groups: int = 1) -> int:
     return int(lib().nvfp4pt_requantize_workspace_bytes(rows, cols, groups))
 
@@ -195,28 +253,32 @@ def requantize_colwise(q_row: torch.Tensor, sf_row: torch.Tensor, amax_row: torc
     """nvfp4pt_requantize_colwise: the columnwise outputs (q_col, sf_col, amax_col) of the
     cast of the dequantized rowwise data; offsets: None or the host row offsets of the
     token groups."""
-    for t, n in ((q_row, "q_row"), (sf_row, "sf_row"), (amax_row, "amax_row")):
-        if not t.is_cuda:
-            raise ValueError(f"{n} must be a CUDA tensor")
+    _require_2d(q_row, "q_row", torch.uint8)
     rows, half = q_row.shape
     cols = 2 * half
+    dev = q_row.get_device()
+    ps = _buf(sf_row, "sf_row", torch.uint8, rows * cols // 16, dev)
+    pa = _buf(amax_row, "amax_row", torch.float32, rows, dev)
     G = 1 if offsets is None else len(offsets) - 1
     if out is None:
-        dev = q_row.device
+        d = q_row.device
         if offsets is None:
-            out = {"q_col": torch.empty((cols, rows // 2), dtype=torch.uint8, device=dev),
-                   "sf_col": torch.empty((cols, rows // 16), dtype=torch.uint8, device=dev),
-                   "amax_col": torch.empty(cols, dtype=torch.float32, device=dev)}
+            out = {"q_col": torch.empty((cols, rows // 2), dtype=torch.uint8, device=d),
+                   "sf_col": torch.empty((cols, rows // 16), dtype=torch.uint8, device=d),
+                   "amax_col": torch.empty(cols, dtype=torch.float32, device=d)}
         else:
-            out = {"q_col": torch.empty(cols * rows // 2, dtype=torch.uint8, device=dev),
-                   "sf_col": torch.empty(cols * rows // 16, dtype=torch.uint8, device=dev),
-                   "amax_col": torch.empty((G, cols), dtype=torch.float32, device=dev)}
+            out = {"q_col": torch.empty(cols * rows // 2, dtype=torch.uint8, device=d),
+                   "sf_col": torch.empty(cols * rows // 16, dtype=torch.uint8, device=d),
+                   "amax_col": torch.empty((G, cols), dtype=torch.float32, device=d)}
     if workspace is None:
         workspace = torch.empty(requantize_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=q_row.device)
+    p = _out_ptrs(out, COLWISE, rows, cols, max(G, 1), dev)
+    pb = _opt_buf(absmax, "absmax", torch.float32, max(G, 1), dev)
+    pw = _buf(workspace, "workspace", torch.uint8, requantize_workspace_bytes(rows, cols, max(G, 1)), dev)
+    _require_cuda(q_row, "q_row")
     off = None if offsets is None else (ctypes.c_int64 * len(offsets))(*[int(o) for o in offsets])
-    st = lib().nvfp4pt_requantize_colwise(
-        _ptr(q_row), _ptr(sf_row), _ptr(amax_row), rows, cols, off, G, _ptr(out["q_col"]), _ptr(out["sf_col"]),
-        _ptr(out["amax_col"]), _ptr(absmax), ctypes.c_float(decay), _ptr(workspace), _stream(stream, q_row.device))
+    st = lib().nvfp4pt_requantize_colwise(_ptr(q_row), ps, pa, rows, cols, off, G, p[3], p[4], p[5], pb,
+                                          ctypes.c_float(decay), pw, _stream(stream, q_row.device))
     _check("nvfp4pt_requantize_colwise", st)
     return out
 
@@ -225,16 +287,19 @@ def quantize_grouped(x: torch.Tensor, offsets, flags: int = ROWWISE | COLWISE, a
                      decay: float = 0.0, out: dict | None = None, workspace: torch.Tensor | None = None,
                      stream: torch.cuda.Stream | None = None) -> dict:
     """nvfp4pt_quantize_grouped. offsets: host sequence of num_groups+1 row offsets."""
-    _require_cuda_bf16(x, "x")
+    _require_2d(x, "x", torch.bfloat16)
     rows, cols = x.shape
+    dev = x.get_device()
     off = (ctypes.c_int64 * len(offsets))(*[int(o) for o in offsets])
     G = len(offsets) - 1
     out = _outputs(rows, cols, flags, x.device, col_rows=rows, groups=G) if out is None else out
     ws = new_workspace(rows, cols, max(G, 1), x.device) if workspace is None else workspace
-    st = lib().nvfp4pt_quantize_grouped(
-        _ptr(x), rows, cols, off, G, flags, _ptr(out.get("q_row")), _ptr(out.get("sf_row")),
-        _ptr(out.get("amax_row")), _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("amax_col")),
-        _ptr(absmax), ctypes.c_float(decay), _ptr(ws), _stream(stream, x.device))
+    p = _out_ptrs(out, flags, rows, cols, max(G, 1), dev)
+    pa = _opt_buf(absmax, "absmax", torch.float32, max(G, 1), dev)
+    pw = _buf(ws, "workspace", torch.uint8, workspace_bytes(rows, cols, max(G, 1)), dev)
+    _require_cuda(x, "x")
+    st = lib().nvfp4pt_quantize_grouped(_ptr(x), rows, cols, off, G, flags, *p, pa, ctypes.c_float(decay), pw,
+                                        _stream(stream, x.device))
     _check("nvfp4pt_quantize_grouped", st)
     return out
 
@@ -242,12 +307,15 @@ def quantize_grouped(x: torch.Tensor, offsets, flags: int = ROWWISE | COLWISE, a
 def quantize_weight_2d(w: torch.Tensor, out: dict | None = None, workspace: torch.Tensor | None = None,
                        stream: torch.cuda.Stream | None = None) -> dict:
     """nvfp4pt_quantize_weight_2d (rowwise outputs with 16x16-block scales)."""
-    _require_cuda_bf16(w, "w")
+    _require_2d(w, "w", torch.bfloat16)
     rows, cols = w.shape
+    dev = w.get_device()
     out = _outputs(rows, cols, ROWWISE, w.device) if out is None else out
     ws = new_workspace(rows, cols, 1, w.device) if workspace is None else workspace
-    st = lib().nvfp4pt_quantize_weight_2d(_ptr(w), rows, cols, _ptr(out["q_row"]), _ptr(out["sf_row"]),
-                                          _ptr(out["amax_row"]), _ptr(ws), _stream(stream, w.device))
+    p = _out_ptrs(out, ROWWISE, rows, cols, 1, dev)
+    pw = _buf(ws, "workspace", torch.uint8, workspace_bytes(rows, cols, 1), dev)
+    _require_cuda(w, "w")
+    st = lib().nvfp4pt_quantize_weight_2d(_ptr(w), rows, cols, p[0], p[1], p[2], pw, _stream(stream, w.device))
     _check("nvfp4pt_quantize_weight_2d", st)
     return out
 
@@ -255,10 +323,11 @@ def quantize_weight_2d(w: torch.Tensor, out: dict | None = None, workspace: torc
 def update_absmax(absmax: torch.Tensor, amax_vec: torch.Tensor, decay: float,
                   stream: torch.cuda.Stream | None = None) -> torch.Tensor:
     """nvfp4pt_update_absmax: absmax[0] = max(absmax[0] * decay, max(amax_vec)), in place."""
-    if not (absmax.is_cuda and amax_vec.is_cuda) or absmax.dtype != torch.float32 or amax_vec.dtype != torch.float32:
-        raise TypeError("absmax and amax_vec must be fp32 CUDA tensors")
-    st = lib().nvfp4pt_update_absmax(_ptr(absmax), _ptr(amax_vec), amax_vec.numel(), ctypes.c_float(decay),
-                                     _stream(stream, absmax.device))
+    dev = absmax.get_device() if isinstance(absmax, torch.Tensor) else -1
+    pb = _buf(absmax, "absmax", torch.float32, 1, dev)
+    pv = _buf(amax_vec, "amax_vec", torch.float32, 0, dev)
+    _require_cuda(absmax, "absmax")
+    st = lib().nvfp4pt_update_absmax(pb, pv, amax_vec.numel(), ctypes.c_float(decay), _stream(stream, absmax.device))
     _check("nvfp4pt_update_absmax", st)
     return absmax
 
@@ -266,7 +335,10 @@ def update_absmax(absmax: torch.Tensor, amax_vec: torch.Tensor, decay: float,
 def workspace_error(workspace: torch.Tensor, stream: torch.cuda.Stream | None = None) -> int:
     """The device error word of the last call on this workspace (synchronises the stream)."""
     word = ctypes.c_uint32(0)
-    st = lib().nvfp4pt_workspace_error(_ptr(workspace), ctypes.byref(word), _stream(stream, workspace.device))
+    dev = workspace.get_device() if isinstance(workspace, torch.Tensor) else -1
+    pw = _buf(workspace, "workspace", torch.uint8, 4, dev)
+    _require_cuda(workspace, "workspace")
+    st = lib().nvfp4pt_workspace_error(pw, ctypes.byref(word), _stream(stream, workspace.device))
     if st not in (0, 8):
         _check("nvfp4pt_workspace_error", st)
     return int(word.value)

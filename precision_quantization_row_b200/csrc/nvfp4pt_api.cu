@@ -102,7 +102,6 @@ nvfp4pt_status encode_map(CUtensorMap* map, const void* x, int64_t rows, int64_t
     return r == CUDA_SUCCESS ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 
-// Workspace layout: [0, 4) error word; [16, ...) observed maxima, one per buffer.
 // Workspace layout: the error word at 0, the observed maxima (one float per group) at
 // 16, then -- in a full workspace -- the row pass's bf16 column maxima [G, cols].
 int64_t pad4(int64_t n) { return (n + 3) & ~int64_t(3); }
