@@ -20,6 +20,14 @@ import oracle
 
 ROWWISE, COLWISE = 1, 2
 
+# Scratch files of the oracle's worker pool live inside the repository (git-ignored).
+_SCRATCH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), ".test_scratch")
+
+
+def _scratch_dir() -> tempfile.TemporaryDirectory:
+    os.makedirs(_SCRATCH, exist_ok=True)
+    return tempfile.TemporaryDirectory(dir=_SCRATCH)
+
 
 def to_np(out: dict) -> dict:
     return {k: v.detach().cpu().numpy() for k, v in out.items()}
@@ -79,7 +87,7 @@ def oracle_quantize_parallel(x: torch.Tensor, flags=ROWWISE | COLWISE, offsets=N
     M, K = xb.shape
     parts = parts or max(1, min(32, os.cpu_count() or 1)) * 2
     out = {"amax_row": np.zeros(M, np.float32)}
-    with tempfile.TemporaryDirectory() as d:
+    with _scratch_dir() as d:
         path = os.path.join(d, "x.npy")
         np.save(path, xb)
         tasks = [("rows", path, a, b, None) for a, b in _split(M, parts)]
@@ -128,7 +136,7 @@ def oracle_weight_2d_parallel(w: torch.Tensor, parts=None) -> dict:
     parts = parts or max(1, min(32, os.cpu_count() or 1)) * 2
     out = {"q_row": np.zeros((N, K // 2), np.uint8), "sf_row": np.zeros((N, K // 16), np.uint8),
            "amax_row": np.zeros(N, np.float32)}
-    with tempfile.TemporaryDirectory() as d:
+    with _scratch_dir() as d:
         path = os.path.join(d, "w.npy")
         np.save(path, wb)
         tasks = [("w2d", path, a, b, None) for a, b in _split(N, parts)]
@@ -137,3 +145,42 @@ def oracle_weight_2d_parallel(w: torch.Tensor, parts=None) -> dict:
                 for k in out:
                     out[k][a:b] = r[k]
     return out
+
+
+# Canary bytes around device buffers: the stand-in for a memory sanitizer (none runs on
+# the GPU pool). Each buffer sits inside a larger uint8 allocation with GUARD bytes of
+# CANARY on each side; a write outside the buffer changes one of them.
+GUARD = 256      # bytes on each side; keeps the buffer 256-byte aligned
+CANARY = 0xA5
+
+
+def guarded(shape, dtype, device) -> tuple:
+    """(raw, view): `view` is a contiguous `dtype` tensor of `shape` inside `raw`."""
+    n = int(np.prod(shape, dtype=np.int64)) * torch.empty((), dtype=dtype).element_size()
+    raw = torch.full((2 * GUARD + n,), CANARY, dtype=torch.uint8, device=device)
+    return raw, raw[GUARD:GUARD + n].view(dtype).view(tuple(shape))
+
+
+def canaries_intact(raw: torch.Tensor) -> bool:
+    r = raw.detach().cpu()
+    return bool((r[:GUARD] == CANARY).all()) and bool((r[-GUARD:] == CANARY).all())
+
+
+def guarded_outputs(rows: int, cols: int, flags: int, device, groups: int = 1) -> tuple:
+    """([raw, ...], out): the cast's output dict (the binding's shapes) in guarded buffers."""
+    shapes = {}
+    if flags & ROWWISE:
+        shapes.update(q_row=((rows, cols // 2), torch.uint8), sf_row=((rows, cols // 16), torch.uint8),
+                      amax_row=((rows,), torch.float32))
+    if flags & COLWISE:
+        if groups == 1:
+            shapes.update(q_col=((cols, rows // 2), torch.uint8), sf_col=((cols, rows // 16), torch.uint8),
+                          amax_col=((cols,), torch.float32))
+        else:
+            shapes.update(q_col=((cols * rows // 2,), torch.uint8), sf_col=((cols * rows // 16,), torch.uint8),
+                          amax_col=((groups, cols), torch.float32))
+    raws, out = [], {}
+    for k, (shape, dtype) in shapes.items():
+        raw, out[k] = guarded(shape, dtype, device)
+        raws.append(raw)
+    return raws, out
