@@ -73,7 +73,7 @@ def test_quantize_rejections(L):
     assert q(P(), 16, 16, 1, None, P(), P(), None, None, None) == 1            # rowwise output missing
     assert q(P(), 16, 16, 2, P(), P(), P(), P(), None, P()) == 1                # colwise output missing
     assert L.nvfp4pt_quantize(P(), 16, 16, 3, *ok7, None, F0, None, None) == 1  # workspace
-    for r, c in [(15, 16), (16, 8), (0, 16), (16, -16), (1 << 31, 16)]:
+    for r, c in [(15, 16), (16, 8), (0, 16), (16, -16), (1 << 31, 16), (96, 70), (70, 96)]:
         assert q(P(), r, c, 3, *ok7) == 2, (r, c)
     for fl in (0, 4, 7):
         assert q(P(), 16, 16, fl, *ok7) == 7, fl
