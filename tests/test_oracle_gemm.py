@@ -155,3 +155,37 @@ def test_rejections(orc):
     with pytest.raises(ValueError):
         orc.gemm_per_token(np.zeros((2, 4), np.uint8), np.zeros((2, 0), np.uint8), a,
                            np.zeros((2, 4), np.uint8), np.zeros((2, 0), np.uint8), a)   # K = 8
+
+
+def test_sum_is_exact_where_a_double_accumulation_rounds(orc):
+    """K = 8192: 511 blocks of codes 6 at scale 448 push the running sum to about 2^55.8
+    units of 2^-20; a last block of +-0.5 and +-1.5 at subnormal scales adds terms of a
+    few units, which a double accumulation rounds away (checked here on the same data).
+    The oracle must equal the exact integer sum (Python integers), rounded once."""
+    rng = np.random.default_rng(97)
+    M, N, K = 2, 3, 8192
+    nb = K // 16
+
+    def operand(R):
+        codes = np.full((R, K), 7)                                    # 6.0
+        codes[:, K - 16:] = rng.choice([1, 3, 9, 11], (R, 16))       # +-0.5, +-1.5
+        sf = np.full((R, nb), 0x7E)                                   # 448
+        sf[:, nb - 1] = rng.integers(1, 8, R)                         # subnormal: m * 2^-9
+        return codes, sf
+
+    (ca, sa), (cb, sb) = operand(M), operand(N)
+    aa, ab = np.full(M, 2688.0, F32), np.full(N, 2688.0, F32)   # decode scale 1
+    d, _ = orc.gemm_per_token(_pack(ca), sa.astype(np.uint8), aa, _pack(cb), sb.astype(np.uint8), ab)
+    twice = [0, 1, 2, 3, 4, 6, 8, 12]
+    sf512 = [int(_e4m3_value(c) * 512) for c in range(0x7F)]
+    for m in range(M):
+        for n in range(N):
+            units, as_double = 0, 0.0   # in 2^-20
+            for k in range(K):
+                va, vb = twice[ca[m, k] & 7], twice[cb[n, k] & 7]
+                t = (-va if ca[m, k] & 8 else va) * (-vb if cb[n, k] & 8 else vb)
+                t *= sf512[sa[m, k // 16]] * sf512[sb[n, k // 16]]
+                units += t
+                as_double += t
+            assert abs(units) > 2 ** 53 and as_double != units   # the regime where doubles round
+            assert d[m, n] == float(Fraction(units, 2 ** 20)), (m, n)
