@@ -6,7 +6,7 @@ import torch
 
 import precision_quantization_row_b200 as nv
 from precision_quantization_row_b200 import inputs
-from parity_util import compare, to_np
+from parity_util import compare, oracle_quantize_parallel, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -122,3 +122,22 @@ def test_requant_of_lossless_rows_equals_direct_cast():
     direct = nv.quantize(x, flags=nv.COLWISE)
     for k in ("q_col", "sf_col", "amax_col"):
         assert torch.equal(got[k].reshape(-1), direct[k].reshape(-1)), k
+
+
+@pytest.mark.slow
+def test_dequant_and_requant_at_the_benchmark_size(orc):
+    """The LLM activation (16384 x 8192) in the launch configuration the benchmark times
+    for both ops: the dequantization against the oracle's, and the columnwise
+    requantization against the oracle's columnwise cast of the dequantized matrix
+    (computed over exact column ranges in parallel)."""
+    x = inputs.llm()
+    r = nv.quantize(x.cuda(), flags=nv.ROWWISE)
+    q, sf, a = (r[k].cpu().numpy() for k in ("q_row", "sf_row", "amax_row"))
+    xd = orc.dequantize(q, sf, a)
+    got = nv.dequantize(r["q_row"], r["sf_row"], r["amax_row"])
+    bad = np.argwhere(got.cpu().view(torch.int16).numpy().view(np.uint16) != xd)
+    assert bad.size == 0, f"{bad.shape[0]} mismatches, first {bad[:3].tolist()}"
+    del got
+    want = oracle_quantize_parallel(torch.from_numpy(xd.view(np.int16)).view(torch.bfloat16), flags=nv.COLWISE)
+    got = nv.requantize_colwise(r["q_row"], r["sf_row"], r["amax_row"])
+    compare(to_np(got), want, label="requant 16384x8192")
