@@ -215,10 +215,18 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_update_absmax(float* absmax_buf, const float*
  * call allocates nothing (no cudaMalloc, no allocating library routine).
  *   - num_groups above NVFP4PT_NOALLOC_MAX_GROUPS (what the array holds) returns
  *     NVFP4PT_ERR_GROUPS before anything is launched.
+ *   - Argument errors are reported exactly as nvfp4pt_quantize_grouped reports them,
+ *     before any CUDA call (no device is touched for a rejected call).
  *   - The first call on a device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current), and so does the first call after the device's context was replaced
+ *     (cudaDeviceReset); make those calls before any stream capture.
  *   - Every call shares the array and clears what it accumulates at its start; calls
  *     that overlap on the GPU (different streams, or different host threads) race on it.
+ *   - The device error word sits in the library's array, where no caller can read it:
+ *     a bounded wait that gives up inside a kernel (only the TMA tile path, taken for
+ *     rows wider than 16384 elements, has such waits) is not reported by this entry;
+ *     the outputs of such a call are then incomplete. Callers that need that report use
+ *     nvfp4pt_quantize_grouped with a workspace and nvfp4pt_workspace_error.
  */
 #define NVFP4PT_NOALLOC_SCRATCH_BYTES 1024
 #define NVFP4PT_NOALLOC_MAX_GROUPS 252

@@ -21,6 +21,7 @@ import torch
 ROWWISE = 1
 COLWISE = 2
 MAX_GROUPS = 1024
+NOALLOC_MAX_GROUPS = 252   # NVFP4PT_NOALLOC_MAX_GROUPS
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnvfp4pt.so")
@@ -34,9 +35,7 @@ STATUS = {
 EXPORTS = (
     "nvfp4pt_status_string", "nvfp4pt_workspace_bytes", "nvfp4pt_quantize", "nvfp4pt_quantize_grouped",
     "nvfp4pt_quantize_weight_2d", "nvfp4pt_update_absmax", "nvfp4pt_workspace_error",
-    "nvfp4pt_probe_transitions", "nvfp4pt_probe_pairs", "nvfp4pt_probe_e4m3_decode", "nvfp4pt_probe_div6",
-    "nvfp4pt_probe_e4m3_div", "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_probe_pair_scales",
-    "nvfp4pt_quantize_timed", "nvfp4pt_dequantize", "nvfp4pt_requantize_workspace_bytes",
+    "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_quantize_timed", "nvfp4pt_dequantize", "nvfp4pt_requantize_workspace_bytes",
     "nvfp4pt_requantize_colwise",
 )
 
@@ -66,13 +65,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_quantize_weight_2d.argtypes = [P, I64, I64, P, P, P, P, P]
         L.nvfp4pt_update_absmax.argtypes = [P, P, I64, F, P]
         L.nvfp4pt_workspace_error.argtypes = [P, P, P]
-        L.nvfp4pt_probe_transitions.argtypes = [I, P, ctypes.c_uint32, P, P]
-        L.nvfp4pt_probe_pairs.argtypes = [P, I64, P, P]
-        L.nvfp4pt_probe_e4m3_decode.argtypes = [P, P]
-        L.nvfp4pt_probe_div6.argtypes = [P, P]
-        L.nvfp4pt_probe_e4m3_div.argtypes = [I, I, P, P]
         L.nvfp4pt_quantize_grouped_noalloc.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, F, P]
-        L.nvfp4pt_probe_pair_scales.argtypes = [I, I, ctypes.c_uint32, P, P]
         L.nvfp4pt_quantize_timed.argtypes = [P, I64, I64, I, P, P, P, P, P, P, P, F, P, P, P]
         L.nvfp4pt_dequantize.argtypes = [P, P, P, I64, I64, P, P]
         L.nvfp4pt_requantize_workspace_bytes.argtypes = [I64, I64, I]
@@ -301,6 +294,27 @@ def quantize_grouped(x: torch.Tensor, offsets, flags: int = ROWWISE | COLWISE, a
     st = lib().nvfp4pt_quantize_grouped(_ptr(x), rows, cols, off, G, flags, *p, pa, ctypes.c_float(decay), pw,
                                         _stream(stream, x.device))
     _check("nvfp4pt_quantize_grouped", st)
+    return out
+
+
+def quantize_grouped_noalloc(x: torch.Tensor, offsets, flags: int = ROWWISE | COLWISE,
+                             absmax: torch.Tensor | None = None, decay: float = 0.0, out: dict | None = None,
+                             stream: torch.cuda.Stream | None = None) -> dict:
+    """nvfp4pt_quantize_grouped_noalloc: the grouped cast without a workspace (its scratch
+    is a static array in the library; at most NOALLOC_MAX_GROUPS token groups). The
+    outputs are allocated here when `out` is None; pass `out` to allocate nothing."""
+    _require_2d(x, "x", torch.bfloat16)
+    rows, cols = x.shape
+    dev = x.get_device()
+    off = (ctypes.c_int64 * len(offsets))(*[int(o) for o in offsets])
+    G = len(offsets) - 1
+    out = _outputs(rows, cols, flags, x.device, col_rows=rows, groups=G) if out is None else out
+    p = _out_ptrs(out, flags, rows, cols, max(G, 1), dev)
+    pa = _opt_buf(absmax, "absmax", torch.float32, max(G, 1), dev)
+    _require_cuda(x, "x")
+    st = lib().nvfp4pt_quantize_grouped_noalloc(_ptr(x), rows, cols, off, G, flags, *p, pa, ctypes.c_float(decay),
+                                                _stream(stream, x.device))
+    _check("nvfp4pt_quantize_grouped_noalloc", st)
     return out
 
 

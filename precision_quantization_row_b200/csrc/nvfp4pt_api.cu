@@ -439,20 +439,21 @@ namespace nvfp4pt {
 
 size_t small_workspace_bytes(int num_groups) { return (size_t)ws_small_bytes(num_groups < 1 ? 1 : num_groups); }
 
-nvfp4pt_status quantize_grouped_ws(const void* x, int64_t rows, int64_t cols, const int64_t* offsets,
-                                   int num_groups, int flags, uint8_t* q_row, uint8_t* sf_row, float* amax_row,
-                                   uint8_t* q_col, uint8_t* sf_col, float* amax_col, float* absmax_bufs, float decay,
-                                   void* workspace, cudaStream_t stream, bool full_ws)
+nvfp4pt_status check_grouped_args(const void* x, int64_t rows, int64_t cols, const int64_t* offsets, int num_groups,
+                                  int flags, const uint8_t* q_row, const uint8_t* sf_row, const float* amax_row,
+                                  const uint8_t* q_col, const uint8_t* sf_col, const float* amax_col,
+                                  const float* absmax_bufs, const void* workspace, bool need_workspace)
 {
     const bool do_row = (flags & NVFP4PT_ROWWISE) != 0;
     const bool do_col = (flags & NVFP4PT_COLWISE) != 0;
-    if (!x || !workspace || !offsets || (do_row && (!q_row || !sf_row || !amax_row)) ||
+    if (!x || (need_workspace && !workspace) || !offsets || (do_row && (!q_row || !sf_row || !amax_row)) ||
         (do_col && (!q_col || !sf_col || !amax_col)))
         return NVFP4PT_ERR_NULL;
     nvfp4pt_status st = check_shape(rows, cols);
     if (st != NVFP4PT_OK) return st;
     if (flags & ~(NVFP4PT_ROWWISE | NVFP4PT_COLWISE) || !(do_row || do_col)) return NVFP4PT_ERR_FLAGS;
-    if (!aligned16(x) || !aligned16(static_cast<uint8_t*>(workspace)) || (absmax_bufs && !aligned16(absmax_bufs)) ||
+    if (!aligned16(x) || (need_workspace && !aligned16(static_cast<const uint8_t*>(workspace))) ||
+        (absmax_bufs && !aligned16(absmax_bufs)) ||
         (do_row && (!aligned16(q_row) || !aligned16(sf_row) || !aligned16(amax_row))) ||
         (do_col && (!aligned16(q_col) || !aligned16(sf_col) || !aligned16(amax_col))))
         return NVFP4PT_ERR_ALIGN;
@@ -460,6 +461,23 @@ nvfp4pt_status quantize_grouped_ws(const void* x, int64_t rows, int64_t cols, co
         return NVFP4PT_ERR_GROUPS;
     for (int g = 0; g < num_groups; ++g)
         if (offsets[g + 1] < offsets[g] || offsets[g] % 16) return NVFP4PT_ERR_GROUPS;
+    return NVFP4PT_OK;
+}
+
+nvfp4pt_status check_device()
+{
+    DeviceState* dev = nullptr;
+    return device_state(&dev);
+}
+
+nvfp4pt_status quantize_grouped_ws(const void* x, int64_t rows, int64_t cols, const int64_t* offsets,
+                                   int num_groups, int flags, uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                   uint8_t* q_col, uint8_t* sf_col, float* amax_col, float* absmax_bufs, float decay,
+                                   void* workspace, cudaStream_t stream, bool full_ws)
+{
+    const nvfp4pt_status st = check_grouped_args(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row,
+                                                 q_col, sf_col, amax_col, absmax_bufs, workspace, true);
+    if (st != NVFP4PT_OK) return st;
     return run_cast<kMaxGroups>(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row, q_col, sf_col,
                                 amax_col, absmax_bufs, decay, false, workspace, stream, nullptr, full_ws);
 }

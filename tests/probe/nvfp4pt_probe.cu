@@ -1,4 +1,4 @@
-// Diagnostic kernels (include/nvfp4pt_probe.h): the cast's device conversions run
+// Diagnostic kernels (nvfp4pt_probe.h, a test-only library): the cast's device conversions run
 // over whole input domains so the tests can compare them with the CPU definition.
 #include "nvfp4pt_probe.h"
 #include "nvfp4pt_device.cuh"

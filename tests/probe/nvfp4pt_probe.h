@@ -1,5 +1,6 @@
 /*
- * nvfp4pt_probe.h -- diagnostic entry points of libnvfp4pt for the test-suite.
+ * nvfp4pt_probe.h -- diagnostic entry points of the test-only libnvfp4pt_probe.so
+ * (built apart from libnvfp4pt.so, which exports only the cast).
  *
  * They run the exact device functions the cast kernels use (the hardware E2M1/E4M3
  * conversions, the E4M3 decode and the correctly rounded division by 6) over whole

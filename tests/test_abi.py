@@ -3,6 +3,7 @@ declare, and rejects bad arguments on the host before touching CUDA."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -18,20 +19,40 @@ def L():
     return nv.lib()
 
 
-def _declared():
+def _declared(paths):
     names = []
-    for h in ("nvfp4pt.h", "nvfp4pt_probe.h", "nvfp4pt_timing.h"):
-        with open(os.path.join(ROOT, "include", h)) as f:
+    for path in paths:
+        with open(path) as f:
             names += re.findall(r"NVFP4PT_API\s+[\w\s\*]+?\b(nvfp4pt_\w+)\s*\(", f.read())
     return names
 
 
+def _exported(lib_path):
+    """Names of the dynamic symbols a shared library defines (nm -D --defined-only)."""
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], check=True, capture_output=True, text=True).stdout
+    return {line.split()[-1] for line in out.splitlines() if line.strip()}
+
+
 def test_every_declared_symbol_is_exported(L):
-    names = _declared()
+    names = _declared([os.path.join(ROOT, "include", h) for h in ("nvfp4pt.h", "nvfp4pt_timing.h")])
     assert len(names) >= 11
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(nv.EXPORTS)
+    # the product library exports the C ABI of the headers and nothing else of ours
+    ours = {s for s in _exported(nv.LIB_PATH) if s.startswith("nvfp4pt")}
+    assert ours == set(names)
+
+
+def test_probe_library_exports_apart():
+    """The diagnostic probes live in their own test-only library."""
+    import probe
+    lib_path = probe.build()
+    names = _declared([os.path.join(ROOT, "tests", "probe", "nvfp4pt_probe.h")])
+    assert set(names) == set(probe.EXPORTS)
+    ours = {s for s in _exported(lib_path) if s.startswith("nvfp4pt")}
+    assert ours == set(names)
+    assert not any(n.startswith("nvfp4pt_probe") for n in _exported(nv.LIB_PATH))
 
 
 def test_status_strings(L):
@@ -149,12 +170,50 @@ def test_dequant_and_requant_rejections(L):
     assert r(offs=[0, 0, 32, 64], G=3) in (5, 6)
 
 
-def test_probe_rejections(L):
+def test_probe_rejections():
+    import probe
+    PL = probe.lib()
     h = _Host()
     P = h.p
-    assert L.nvfp4pt_probe_transitions(0, None, 8, P(), None) == 1
-    assert L.nvfp4pt_probe_transitions(2, P(), 8, P(), None) == 7
-    assert L.nvfp4pt_probe_pairs(P(), 0, P(), None) == 2
+    assert PL.nvfp4pt_probe_transitions(0, None, 8, P(), None) == 1
+    assert PL.nvfp4pt_probe_transitions(2, P(), 8, P(), None) == 7
+    assert PL.nvfp4pt_probe_pairs(P(), 0, P(), None) == 2
+
+
+def test_noalloc_rejections(L):
+    """The entry without allocation reports argument errors as the grouped cast does,
+    before any CUDA call (here, on a machine without a GPU, nothing else can run)."""
+    h = _Host()
+    P = h.p
+
+    def n(offs=(0, 64), G=None, rows=64, cols=32, flags=3, outs=None, x=None, bufs=None):
+        arr = None if offs is None else (ctypes.c_int64 * len(offs))(*offs)
+        G = len(offs) - 1 if G is None else G
+        o = [P()] * 6 if outs is None else outs
+        return L.nvfp4pt_quantize_grouped_noalloc(P() if x is None else x, rows, cols, arr, G, flags, *o, bufs, F0,
+                                                  None)
+
+    assert L.nvfp4pt_quantize_grouped_noalloc(None, 64, 32, (ctypes.c_int64 * 2)(0, 64), 1, 3, *[P()] * 6, None,
+                                              F0, None) == 1
+    assert n(offs=None, G=1) == 1
+    assert n(flags=1, outs=[None, P(), P(), None, None, None]) == 1      # rowwise output missing
+    assert n(flags=2, outs=[None, None, None, P(), P(), None]) == 1      # colwise output missing
+    for r, c in [(15, 16), (16, 8), (0, 16), (1 << 31, 16), (96, 70)]:
+        assert n(offs=(0, max(r, 0)), rows=r, cols=c) == 2, (r, c)
+    for fl in (0, 4, 7):
+        assert n(flags=fl) == 7, fl
+    assert n(x=P(8)) == 3
+    assert n(outs=[P(4), P(), P(), P(), P(), P()]) == 3
+    assert n(bufs=P(4)) == 3
+    assert n(offs=(0, 64), G=0) == 4
+    assert n(offs=(16, 64)) == 4
+    assert n(offs=(0, 32, 16, 64)) == 4
+    assert n(offs=(0, 8, 64)) == 4
+    # more groups than the static array holds (NVFP4PT_NOALLOC_MAX_GROUPS = 252)
+    offs = tuple(range(0, 16 * 253 + 1, 16))
+    assert n(offs=offs, rows=16 * 253) == 4
+    # valid arguments pass validation and fail only at the device step here
+    assert n(offs=(0, 0, 32, 64)) in (5, 6)
 
 
 def test_binding_refuses_cpu_tensors():

@@ -55,6 +55,21 @@ def test_grouped_cast():
     _check(raws + [ws_raw, b_raw], dict(out, absmax=bufs), dict(want, absmax=ref_bufs))
 
 
+@pytest.mark.parametrize("cols", [272, 16400], ids=["row_pass", "tile_path"])
+def test_grouped_cast_noalloc(cols):
+    """The entry without allocation: guarded outputs and buffers, the same bytes as the
+    workspace entry on plain buffers."""
+    rows, G = 400, len(OFFSETS) - 1
+    x = inputs.random_shape(85, rows, cols, "wide").cuda()
+    raws, out = guarded_outputs(rows, cols, nv.ROWWISE | nv.COLWISE, "cuda", groups=G)
+    b_raw, bufs = guarded((G,), torch.float32, "cuda")
+    bufs.fill_(2.0)
+    nv.quantize_grouped_noalloc(x, OFFSETS, absmax=bufs, decay=0.5, out=out)
+    ref_bufs = torch.full((G,), 2.0, dtype=torch.float32, device="cuda")
+    want = nv.quantize_grouped(x, OFFSETS, absmax=ref_bufs, decay=0.5)
+    _check(raws + [b_raw], dict(out, absmax=bufs), dict(want, absmax=ref_bufs))
+
+
 @pytest.mark.parametrize("shape", [(144, 272), (64, 16400)], ids=lambda s: f"{s[0]}x{s[1]}")
 def test_weight_2d(shape):
     rows, cols = shape

@@ -16,7 +16,7 @@ import numpy as np
 import pytest
 import torch
 
-import precision_quantization_row_b200 as nv
+import probe
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ def _transitions(which: int):
     cap = 1 << 16
     out = torch.zeros(2 * cap, dtype=torch.int32, device="cuda")
     cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
-    st = nv.lib().nvfp4pt_probe_transitions(which, ctypes.c_void_p(out.data_ptr()), cap,
+    st = probe.lib().nvfp4pt_probe_transitions(which, ctypes.c_void_p(out.data_ptr()), cap,
                                             ctypes.c_void_p(cnt.data_ptr()),
                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
@@ -66,7 +66,7 @@ def _pairs(lo_hi):
     a = torch.tensor(np.asarray(lo_hi, np.float32).ravel(), device="cuda")
     n = a.numel() // 2
     out = torch.zeros(n, dtype=torch.int32, device="cuda")
-    st = nv.lib().nvfp4pt_probe_pairs(ctypes.c_void_p(a.data_ptr()), n, ctypes.c_void_p(out.data_ptr()),
+    st = probe.lib().nvfp4pt_probe_pairs(ctypes.c_void_p(a.data_ptr()), n, ctypes.c_void_p(out.data_ptr()),
                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     return out.cpu().numpy().view(np.uint32)
@@ -91,7 +91,7 @@ def test_pair_order(orc):
 
 def test_e4m3_decode(orc):
     out = torch.zeros(512, dtype=torch.float32, device="cuda")
-    st = nv.lib().nvfp4pt_probe_e4m3_decode(ctypes.c_void_p(out.data_ptr()),
+    st = probe.lib().nvfp4pt_probe_e4m3_decode(ctypes.c_void_p(out.data_ptr()),
                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     d = out.cpu().numpy()
@@ -105,7 +105,7 @@ def test_e4m3_decode(orc):
 
 def test_div6_exhaustive():
     out = torch.zeros(0x7F80, dtype=torch.float32, device="cuda")
-    st = nv.lib().nvfp4pt_probe_div6(ctypes.c_void_p(out.data_ptr()),
+    st = probe.lib().nvfp4pt_probe_div6(ctypes.c_void_p(out.data_ptr()),
                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     got = out.cpu().numpy().view(np.uint32)
@@ -121,7 +121,7 @@ def test_block_scale_division_matches_ieee(lo, hi):
     binades (down to the smallest possible s_enc, 2688/FLT_MAX ~ 2^-117, where the
     remainder can be subnormal), the middle, and the overflow edge (clamped to FLT_MAX)."""
     bad = torch.zeros(1, dtype=torch.int64, device="cuda")
-    st = nv.lib().nvfp4pt_probe_e4m3_div(lo, hi, ctypes.c_void_p(bad.data_ptr()),
+    st = probe.lib().nvfp4pt_probe_e4m3_div(lo, hi, ctypes.c_void_p(bad.data_ptr()),
                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     assert int(bad.item()) == 0
@@ -133,7 +133,7 @@ def test_packed_block_scales_match_scalar():
     block amax, against every 4093rd significand of s in every binade that s_enc can
     take (2688 / max bf16 ~ 2^-117 up to FLT_MAX), plus s = FLT_MAX and s = 1."""
     bad = torch.zeros(1, dtype=torch.int64, device="cuda")
-    st = nv.lib().nvfp4pt_probe_pair_scales(10, 254, 4093, ctypes.c_void_p(bad.data_ptr()),
+    st = probe.lib().nvfp4pt_probe_pair_scales(10, 254, 4093, ctypes.c_void_p(bad.data_ptr()),
                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     assert int(bad.item()) == 0
