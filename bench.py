@@ -435,6 +435,81 @@ def run_gpu_op(args, dist: Dist, op: str) -> dict | None:
     }
 
 
+def measured_tensor_peak():
+    """Dense FP4 tensor peak: the measured bf16 burst (cuBLAS) times the nominal FP4/bf16
+    ratio 4 (9 and 2.25 PFLOP/s dense), or the fallback bf16 figure times 4."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 4 (nominal fp4/bf16)"
+    except Exception:
+        return 4.0 * 1590.0, "fallback bf16 x 4 (nominal fp4/bf16)"
+
+
+def run_gpu_gemm(args, dist: Dist) -> dict | None:
+    """Device time of nvfp4pt_gemm_per_token on the forward product of the headline layer:
+    A = the rowwise cast of the 16384 x 8192 activation, B = the rowwise cast of an
+    8192 x 8192 weight (N(0, 0.02)), D = A B^T in fp32 (two output buffers rotate)."""
+    import torch
+
+    import precision_quantization_row_b200 as nv
+    from precision_quantization_row_b200 import build, inputs
+
+    build.build()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    stream = torch.cuda.current_stream(dev)
+    m, k, n = args.rows, args.cols, args.gemm_n
+    x = inputs.llm(M=m, K=k).to(dev)
+    g = torch.Generator(device=dev).manual_seed(6)
+    w = (torch.randn((n, k), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    a = nv.quantize(x, flags=nv.ROWWISE)
+    b = nv.quantize(w, flags=nv.ROWWISE)
+    del x, w
+    outs = [torch.empty((m, n), dtype=torch.float32, device=dev) for _ in range(2)]
+    ws = nv.new_gemm_workspace(dev)
+
+    def step(i):
+        nv.gemm_per_token(a["q_row"], a["sf_row"], a["amax_row"], b["q_row"], b["sf_row"], b["amax_row"],
+                          out=outs[i & 1], workspace=ws, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run():
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1) / 1e3
+
+    with ClockSampler(dev.index) as clk:
+        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    if nv.workspace_error(ws) != 0:
+        raise RuntimeError("device error word set during the timed region")
+    if dist.rank != 0:
+        return None
+    peak, peak_kind = measured_tensor_peak()
+    per = secs / args.steps
+    flops = 2.0 * m * n * k
+    tflops = flops / per / 1e12
+    return {
+        "metric": "NVFP4 per-token GEMM (block-scaled tcgen05, amax-vector epilogue): TFLOP/s",
+        "value": flops * args.steps * dist.world / secs / 1e12, "unit": "TFLOP/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 x nvfp4 -> fp32 (e2m1, e4m3 block16 scales)",
+        "data": "synthetic",
+        "config": {"workload": f"gemm_fprop_{m}x{n}x{k}", "m": m, "n": n, "k": k,
+                   "l2": "operands 151 MB, 2 rotating fp32 outputs of " f"{m * n * 4 / 1e6:.0f} MB"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_flops_per_call": flops},
+        "gpu_launches": args.steps, "clocks": clk.summary(),
+    }
+
+
 def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
     """Device time per call of the other workloads (parity-test configurations, reported
     beside the headline): dense 4096x4096 row+column cast, the grouped MoE cast
@@ -579,8 +654,9 @@ def main(argv=None):
     ap.add_argument("--cols", type=int, default=8192, help="columns of the activation (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
-    ap.add_argument("--op", choices=["cast", "dequant", "requant"], default="cast",
-                    help="cast: the per-token cast (the headline); dequant / requant: the secondary ops")
+    ap.add_argument("--op", choices=["cast", "dequant", "requant", "gemm"], default="cast",
+                    help="cast: the per-token cast (the headline); dequant / requant / gemm: the secondary ops")
+    ap.add_argument("--gemm-n", type=int, default=8192, help="N of --op gemm (M = --rows, K = --cols)")
     ap.add_argument("--config", choices=["llm", "dense", "moe", "weight"], default="llm",
                     help="llm: the headline activation; the others time the remaining workloads")
     args = ap.parse_args(argv)
@@ -602,7 +678,7 @@ def main(argv=None):
         return
     if args.op != "cast":
         try:
-            line = run_gpu_op(args, dist, args.op)
+            line = run_gpu_gemm(args, dist) if args.op == "gemm" else run_gpu_op(args, dist, args.op)
             if line is not None:
                 print(json.dumps(line), flush=True)
         finally:

@@ -194,6 +194,40 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, cons
                                                       float* absmax_bufs, float decay, void* workspace,
                                                       cudaStream_t stream);
 
+/* Bytes of the workspace of nvfp4pt_gemm_per_token (its device error word). */
+NVFP4PT_API size_t nvfp4pt_gemm_workspace_bytes(void);
+
+/*
+ * nvfp4pt_gemm_per_token -- the GEMM of two per-token NVFP4 operands, rescaled in its
+ * epilogue by the per-row and per-column outer-amax vectors (TransformerEngine PR #3045
+ * "Add NVFP4 per-token quantization recipe", Description: a CUTLASS GEMM that rescales
+ * with the per-row/per-col outer-amax vectors inside the epilogue; Greptile summary: the
+ * TN forward, NN data-gradient and NT weight-gradient products). The page prints no
+ * formula; the reading taken, with the decode scale S_dec(amax) = RN(amax / 2688) of the
+ * dequantization:
+ *     acc[m][n] = sum_k val(qa[m][k]) * float(sfa[m][k/16]) * val(qb[n][k]) * float(sfb[n][k/16])
+ *     d[m][n]   = RN( RN(acc[m][n] * S_dec(amax_a[m])) * S_dec(amax_b[n]) )
+ * Each 16-element block product is exact in binary32; acc is the tensor cores' fp32
+ * accumulation of them (block-scaled MMAs of 64 elements, summed in K order), so d
+ * differs from the exact value by a few fp32 roundings of the partial sums.
+ * Both operands are K-major rowwise data as nvfp4pt_quantize writes it (the rowwise
+ * data of a matrix, or the columnwise data of its transpose), so all three products are
+ * this one call:
+ *   qa, sfa, amax_a  uint8 [m, k/2] codes, uint8 [m, k/16] E4M3 scales, fp32 [m] amax
+ *   qb, sfb, amax_b  uint8 [n, k/2], uint8 [n, k/16], fp32 [n]
+ *   d                fp32 [m, n] row-major, written in full
+ *   workspace        nvfp4pt_gemm_workspace_bytes() bytes; holds the error word that
+ *                    nvfp4pt_workspace_error reads (a wait inside the kernel that gave up)
+ * Block scales must be non-negative finite E4M3 codes (0x00..0x7E), as the cast writes.
+ * m and n are multiples of 16, k a multiple of 256 (a row of block scales is then a
+ * whole number of 16-byte units, as the tensor-memory-access copies require), all at
+ * most 2^30; pointers 16-byte aligned. Errors as in the casts, before any launch.
+ */
+NVFP4PT_API nvfp4pt_status nvfp4pt_gemm_per_token(const uint8_t* qa, const uint8_t* sfa, const float* amax_a,
+                                                  int64_t m, const uint8_t* qb, const uint8_t* sfb,
+                                                  const float* amax_b, int64_t n, int64_t k, float* d,
+                                                  void* workspace, cudaStream_t stream);
+
 /*
  * nvfp4pt_update_absmax -- the running-buffer step alone (PR #3296, Description):
  * *absmax_buf = max(RN(*absmax_buf * decay), max_i amax_vec[i]); n may be 0

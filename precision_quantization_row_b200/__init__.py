@@ -36,7 +36,7 @@ EXPORTS = (
     "nvfp4pt_status_string", "nvfp4pt_workspace_bytes", "nvfp4pt_quantize", "nvfp4pt_quantize_grouped",
     "nvfp4pt_quantize_weight_2d", "nvfp4pt_update_absmax", "nvfp4pt_workspace_error",
     "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_quantize_timed", "nvfp4pt_dequantize", "nvfp4pt_requantize_workspace_bytes",
-    "nvfp4pt_requantize_colwise",
+    "nvfp4pt_requantize_colwise", "nvfp4pt_gemm_workspace_bytes", "nvfp4pt_gemm_per_token",
 )
 
 
@@ -70,9 +70,12 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_dequantize.argtypes = [P, P, P, I64, I64, P, P]
         L.nvfp4pt_requantize_workspace_bytes.argtypes = [I64, I64, I]
         L.nvfp4pt_requantize_colwise.argtypes = [P, P, P, I64, I64, P, I, P, P, P, P, F, P, P]
+        L.nvfp4pt_gemm_workspace_bytes.argtypes = []
+        L.nvfp4pt_gemm_per_token.argtypes = [P, P, P, I64, P, P, P, I64, I64, P, P, P]
         for name in EXPORTS[2:]:
             getattr(L, name).restype = I
         L.nvfp4pt_requantize_workspace_bytes.restype = ctypes.c_size_t
+        L.nvfp4pt_gemm_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -233,6 +236,45 @@ def dequantize(q: torch.Tensor, sf: torch.Tensor, amax: torch.Tensor, out: torch
     st = lib().nvfp4pt_dequantize(_ptr(q), ps, pa, rows, cols, po, _stream(stream, q.device))
     _check("nvfp4pt_dequantize", st)
     return out
+
+
+def gemm_per_token(qa: torch.Tensor, sfa: torch.Tensor, amax_a: torch.Tensor, qb: torch.Tensor,
+                   sfb: torch.Tensor, amax_b: torch.Tensor, out: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """nvfp4pt_gemm_per_token: D [m, n] fp32 of two K-major rowwise NVFP4 operands (A: q
+    uint8 [m, k/2], sf uint8 [m, k/16], amax fp32 [m]; B likewise with n rows), rescaled by
+    S_dec(amax_a[m]) * S_dec(amax_b[n]) in the epilogue."""
+    _require_2d(qa, "qa", torch.uint8)
+    _require_2d(qb, "qb", torch.uint8)
+    m, half = qa.shape
+    n = qb.shape[0]
+    k = 2 * half
+    if qb.shape[1] != half:
+        raise ValueError(f"qa and qb differ in K: {qa.shape} vs {qb.shape}")
+    dev = qa.get_device()
+    psa = _buf(sfa, "sfa", torch.uint8, m * k // 16, dev)
+    paa = _buf(amax_a, "amax_a", torch.float32, m, dev)
+    pqb = _buf(qb, "qb", torch.uint8, n * k // 2, dev)
+    psb = _buf(sfb, "sfb", torch.uint8, n * k // 16, dev)
+    pab = _buf(amax_b, "amax_b", torch.float32, n, dev)
+    out = torch.empty((m, n), dtype=torch.float32, device=qa.device) if out is None else out
+    po = _buf(out, "out", torch.float32, m * n, dev)
+    ws = new_gemm_workspace(qa.device) if workspace is None else workspace
+    pw = _buf(ws, "workspace", torch.uint8, gemm_workspace_bytes(), dev)
+    _require_cuda(qa, "qa")
+    st = lib().nvfp4pt_gemm_per_token(_ptr(qa), psa, paa, m, pqb, psb, pab, n, k, po, pw,
+                                      _stream(stream, qa.device))
+    _check("nvfp4pt_gemm_per_token", st)
+    return out
+
+
+@functools.lru_cache(maxsize=1)
+def gemm_workspace_bytes() -> int:
+    return int(lib().nvfp4pt_gemm_workspace_bytes())
+
+
+def new_gemm_workspace(device=None) -> torch.Tensor:
+    return torch.empty(gemm_workspace_bytes(), dtype=torch.uint8, device=device)
 
 
 @functools.lru_cache(maxsize=256)

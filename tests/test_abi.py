@@ -170,6 +170,26 @@ def test_dequant_and_requant_rejections(L):
     assert r(offs=[0, 0, 32, 64], G=3) in (5, 6)
 
 
+def test_gemm_rejections(L):
+    h = _Host()
+    P = h.p
+    g = lambda qa=None, m=128, n=256, k=512, d=None, ws=None, sfb=None: L.nvfp4pt_gemm_per_token(
+        P() if qa is None else qa, P(), P(), m, P(), P() if sfb is None else sfb, P(), n, k,
+        P() if d is None else d, P() if ws is None else ws, None)
+    assert L.nvfp4pt_gemm_workspace_bytes() >= 4
+    assert L.nvfp4pt_gemm_per_token(None, P(), P(), 16, P(), P(), P(), 16, 256, P(), P(), None) == 1
+    assert L.nvfp4pt_gemm_per_token(P(), P(), P(), 16, P(), P(), P(), 16, 256, None, P(), None) == 1
+    assert L.nvfp4pt_gemm_per_token(P(), P(), P(), 16, P(), P(), P(), 16, 256, P(), None, None) == 1
+    for m, n, k in [(0, 16, 256), (16, 8, 256), (20, 16, 256), (16, 16, 128), (16, 16, 300), (16, 16, 0),
+                    (1 << 31, 16, 256)]:
+        assert g(m=m, n=n, k=k) == 2, (m, n, k)
+    assert g(qa=P(8)) == 3
+    assert g(sfb=P(4)) == 3
+    assert g(d=P(4)) == 3
+    # valid arguments pass validation and fail only at the device step here
+    assert g() in (5, 6)
+
+
 def test_probe_rejections():
     import probe
     PL = probe.lib()

@@ -107,6 +107,21 @@ def test_requantize(shape, offsets):
     _check(raws + [ws_raw, b_raw], dict(out, absmax=bufs), dict(want, absmax=ref_bufs))
 
 
+def test_gemm():
+    m, n, k = 144, 272, 512
+    g = torch.Generator(device="cuda").manual_seed(86)
+    qa = torch.randint(0, 256, (m, k // 2), dtype=torch.uint8, device="cuda", generator=g)
+    qb = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device="cuda", generator=g)
+    sfa = torch.randint(0, 0x7F, (m, k // 16), dtype=torch.uint8, device="cuda", generator=g)
+    sfb = torch.randint(0, 0x7F, (n, k // 16), dtype=torch.uint8, device="cuda", generator=g)
+    aa = torch.rand(m, device="cuda", generator=g)
+    ab = torch.rand(n, device="cuda", generator=g)
+    d_raw, d = guarded((m, n), torch.float32, "cuda")
+    ws_raw, ws = guarded((nv.gemm_workspace_bytes(),), torch.uint8, "cuda")
+    nv.gemm_per_token(qa, sfa, aa, qb, sfb, ab, out=d, workspace=ws)
+    _check([d_raw, ws_raw], {"d": d}, {"d": nv.gemm_per_token(qa, sfa, aa, qb, sfb, ab)})
+
+
 def test_update_absmax():
     v = torch.rand(1000, dtype=torch.float32, device="cuda") * 3
     b_raw, buf = guarded((1,), torch.float32, "cuda")
