@@ -213,6 +213,87 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+
+# ------------------------------------------------------- timing + baselines
+
+def repeat_count(args, per_region_s: float) -> int:
+    """Timed regions of `steps` steps each: --repeats, else enough for ~1 s of timed work
+    (at least 5, at most 50), so that the median is steady and NVML sees many samples."""
+    if args.repeats > 0:
+        return args.repeats
+    return int(max(5, min(50, 1.0 / max(per_region_s, 1e-6))))
+
+
+def timed_regions(args, dist: Dist, dev, stream, step) -> tuple[float, list, dict]:
+    """Warm-up, then R timed regions of `args.steps` steps each (CUDA events on the
+    launching stream, barrier + sync on both sides, max over ranks), NVML sampled over
+    all of them. Returns (median region seconds, all region seconds, clock summary)."""
+    import torch
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def region():
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1) / 1e3
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    probe = timed_region(dist, region, lambda: torch.cuda.synchronize(dev))
+    reps = repeat_count(args, probe)
+    secs = []
+    with ClockSampler(dev.index) as clk:
+        for _ in range(reps):
+            secs.append(timed_region(dist, region, lambda: torch.cuda.synchronize(dev)))
+    return statistics.median(secs), secs, clk.summary()
+
+
+def region_stats(secs: list) -> dict:
+    ms = sorted(s * 1e3 for s in secs)
+    return {"repeats": len(ms), "region_ms_min": ms[0], "region_ms_median": statistics.median(ms),
+            "region_ms_max": ms[-1]}
+
+
+def cpu_info() -> dict:
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+def pinned(fn):
+    """Run fn() with this process pinned to one core (the first it may use), as
+    `taskset -c <core>` would; returns (fn's result, seconds, core)."""
+    old = os.sched_getaffinity(0)
+    core = min(old)
+    os.sched_setaffinity(0, {core})
+    try:
+        t = time.perf_counter()
+        r = fn()
+        return r, time.perf_counter() - t, core
+    finally:
+        os.sched_setaffinity(0, old)
+
+
+def oracle_baseline(elems: int, run, sample: str, unit_scale=None) -> dict:
+    """The oracle as it stands, single-threaded, pinned to one core, on a bounded sample:
+    `run()` does `elems` elements of the workload's cast."""
+    _, secs, core = pinned(run)
+    d = {"value": elems / secs, "unit": "elem/s", "cores": 1, "kind": "oracle", "sample": sample,
+         "seconds": secs, "pinned_core": core}
+    d.update(cpu_info())
+    return d
+
+
 # --------------------------------------------------------------- GPU arm
 
 def run_gpu(args, dist: Dist) -> dict | None:
@@ -238,24 +319,9 @@ def run_gpu(args, dist: Dist) -> dict | None:
     def step(i):
         nv.quantize(xs[i & 1], absmax=buf, decay=DECAY, out=outs[i & 1], workspace=ws, stream=stream)
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
+    secs, all_secs, clocks = timed_regions(args, dist, dev, stream, step)
     if nv.workspace_error(ws) != 0:
-        raise RuntimeError("device error word set during warm-up")
-
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def run():
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        ev1.synchronize()
-        return ev0.elapsed_time(ev1) / 1e3
-
-    with ClockSampler(dev.index) as clk:
-        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+        raise RuntimeError("device error word set during the timed region")
     launches = nv.CAST_LAUNCHES * args.steps  # zero, row pass, column pass per cast
 
     # Per-kernel times: the same casts through the timed entry, which records an event
@@ -277,38 +343,7 @@ def run_gpu(args, dist: Dist) -> dict | None:
     kernel_ms = {name: dist.max(sum(row[j].elapsed_time(row[j + 1]) for row in kevs) / kt_steps)
                  for j, name in enumerate(KERNELS)}
 
-    # end to end through the public call with host buffers: pinned H2D of the input,
-    # the cast, D2H of every output (codes, scales, amax vectors, buffer)
-    e2e = None
-    if not args.no_e2e:
-        xh = x_host.pin_memory()
-        host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs[0].items()}
-        buf_h = torch.empty(1, dtype=torch.float32, pin_memory=True)
-        h2d = xh.numel() * xh.element_size()
-        d2h = sum(v.numel() * v.element_size() for v in host_out.values()) + buf_h.numel() * 4
-        e2e_steps = max(3, min(args.steps, 10))
-
-        def e2e_step(i):
-            xs[0].copy_(xh, non_blocking=True)
-            nv.quantize(xs[0], absmax=buf, decay=DECAY, out=outs[0], workspace=ws, stream=stream)
-            for k, v in outs[0].items():
-                host_out[k].copy_(v, non_blocking=True)
-            buf_h.copy_(buf, non_blocking=True)
-
-        for i in range(2):
-            e2e_step(i)
-
-        def run_e2e():
-            ev0.record(stream)
-            for i in range(e2e_steps):
-                e2e_step(i)
-            ev1.record(stream)
-            ev1.synchronize()
-            return ev0.elapsed_time(ev1) / 1e3
-
-        e2e_secs = timed_region(dist, run_e2e, lambda: torch.cuda.synchronize(dev))
-        e2e = {"value": float(M) * K * e2e_steps * dist.world / e2e_secs, "unit": "elem/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    e2e = None if args.no_e2e else run_e2e(args, dist, dev, stream, x_host, xs, outs, buf, ws)
     if nv.workspace_error(ws) != 0:
         raise RuntimeError("device error word set during the timed region")
 
@@ -338,6 +373,7 @@ def run_gpu(args, dist: Dist) -> dict | None:
                    "absmax_decay": DECAY, "parallelism": f"replicas x{dist.world}",
                    "l2": f"inputs larger than L2 ({M * K * 2 / 1e6:.0f} MB each), 2 rotating input copies "
                          "and output sets"},
+        "timing": dict(region_stats(all_secs), note="value and ms_per_step: the median region"),
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": kernel_bytes(dominant, M, K),
@@ -350,12 +386,65 @@ def run_gpu(args, dist: Dist) -> dict | None:
                               "algorithmic_bytes_per_cast": algo_bytes(M, K)}},
         "e2e": e2e,
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     return line
 
 
-# ------------------------------------------------------------ oracle arm
+def run_e2e(args, dist: Dist, dev, stream, x_host, xs, outs, buf, ws) -> dict:
+    """The public call end to end with host buffers: every step copies its input from
+    pinned host memory and every output (codes, scales, amax vectors, buffer) back. The
+    copies run on their own streams, two buffer sets deep, so that step i+1's input
+    crosses PCIe while step i's outputs come back (full duplex); the timed region runs
+    from the first copy in to the last copy out."""
+    import torch
+
+    import precision_quantization_row_b200 as nv
+    m, k = x_host.shape
+    xh = x_host.pin_memory()
+    host_out = [{n: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for n, v in outs[0].items()}
+                for _ in range(2)]
+    buf_h = [torch.empty(1, dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    h2d = xh.numel() * xh.element_size()
+    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values()) + 4
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = max(4, min(args.steps, 12))
+    ev_in = [torch.cuda.Event() for _ in range(n)]
+    ev_c = [torch.cuda.Event() for _ in range(n)]
+    ev_out = [torch.cuda.Event() for _ in range(n)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def region():
+        t0.record(s_in)
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(ev_c[i - 2])       # the cast of step i-2 has read xs[b]
+            with torch.cuda.stream(s_in):
+                xs[b].copy_(xh, non_blocking=True)
+            ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])   # step i-2's outputs have left outs[b]
+            nv.quantize(xs[b], absmax=buf, decay=DECAY, out=outs[b], workspace=ws, stream=stream)
+            ev_c[i].record(stream)
+            s_out.wait_event(ev_c[i])
+            with torch.cuda.stream(s_out):
+                for name, v in outs[b].items():
+                    host_out[b][name].copy_(v, non_blocking=True)
+                buf_h[b].copy_(buf, non_blocking=True)
+            ev_out[i].record(s_out)
+        s_out.wait_event(ev_c[n - 1])
+        t1.record(s_out)
+        t1.synchronize()
+        return t0.elapsed_time(t1) / 1e3
+
+    timed_region(dist, region, lambda: torch.cuda.synchronize(dev))   # warm-up of the copy path
+    secs = statistics.median(timed_region(dist, region, lambda: torch.cuda.synchronize(dev)) for _ in range(3))
+    return {"value": float(m) * k * n * dist.world / secs, "unit": "elem/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n,
+            "note": "pinned host buffers; copy-in, cast and copy-out on three streams, two buffer sets deep"}
+
 
 def op_bytes(op: str, m: int, k: int) -> int:
     """Algorithmic bytes of the secondary ops. Dequantize: rowwise codes, scales and
@@ -401,21 +490,7 @@ def run_gpu_op(args, dist: Dist, op: str) -> dict | None:
         # rows up to 16384 wide: the cast's three kernels read the NVFP4 data directly;
         # wider: a dequantize launch first
         launches = nv.CAST_LAUNCHES + (0 if k <= 16384 else 1)
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def run():
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        ev1.synchronize()
-        return ev0.elapsed_time(ev1) / 1e3
-
-    with ClockSampler(dev.index) as clk:
-        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    secs, all_secs, clocks = timed_regions(args, dist, dev, stream, step)
     if dist.rank != 0:
         return None
     peak, peak_kind = measured_peak()
@@ -429,9 +504,10 @@ def run_gpu_op(args, dist: Dist, op: str) -> dict | None:
         "dtype": "nvfp4->bf16" if op == "dequant" else "nvfp4->nvfp4 (bf16 values in registers)", "data": "synthetic",
         "config": {"workload": f"{op}_rowwise_{m}x{k}", "rows": m, "cols": k,
                    "l2": "two rotating input sets and outputs"},
+        "timing": region_stats(all_secs),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": None, "peak_source": peak_kind, "algorithmic_bytes_per_call": op_bytes(op, m, k)},
-        "gpu_launches": launches * args.steps, "clocks": clk.summary(),
+        "gpu_launches": launches * args.steps, "clocks": clocks,
     }
 
 
@@ -472,21 +548,7 @@ def run_gpu_gemm(args, dist: Dist) -> dict | None:
         nv.gemm_per_token(a["q_row"], a["sf_row"], a["amax_row"], b["q_row"], b["sf_row"], b["amax_row"],
                           out=outs[i & 1], workspace=ws, stream=stream)
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def run():
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        ev1.synchronize()
-        return ev0.elapsed_time(ev1) / 1e3
-
-    with ClockSampler(dev.index) as clk:
-        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    secs, all_secs, clocks = timed_regions(args, dist, dev, stream, step)
     if nv.workspace_error(ws) != 0:
         raise RuntimeError("device error word set during the timed region")
     if dist.rank != 0:
@@ -495,7 +557,7 @@ def run_gpu_gemm(args, dist: Dist) -> dict | None:
     per = secs / args.steps
     flops = 2.0 * m * n * k
     tflops = flops / per / 1e12
-    return {
+    line = {
         "metric": "NVFP4 per-token GEMM (block-scaled tcgen05, amax-vector epilogue): TFLOP/s",
         "value": flops * args.steps * dist.world / secs / 1e12, "unit": "TFLOP/s", "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
@@ -503,18 +565,35 @@ def run_gpu_gemm(args, dist: Dist) -> dict | None:
         "data": "synthetic",
         "config": {"workload": f"gemm_fprop_{m}x{n}x{k}", "m": m, "n": n, "k": k,
                    "l2": "operands 151 MB, 2 rotating fp32 outputs of " f"{m * n * 4 / 1e6:.0f} MB"},
+        "timing": region_stats(all_secs),
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "traffic": None, "peak_source": peak_kind,
                      "algorithmic_flops_per_call": flops},
-        "gpu_launches": args.steps, "clocks": clk.summary(),
+        "gpu_launches": args.steps, "clocks": clocks,
     }
+    if not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        cpu = lambda t: t.cpu().numpy()
+        rows = 32
+        A = [cpu(a[n_][:rows]) for n_ in ("q_row", "sf_row", "amax_row")]
+        B = [cpu(b[n_][:rows]) for n_ in ("q_row", "sf_row", "amax_row")]
+        base = oracle_baseline(0, lambda: oracle.gemm_per_token(*A, *B),
+                               f"the exact-sum oracle on the first {rows} rows of A x the first {rows} rows of B "
+                               f"(k = {k})")
+        base["value"] = 2.0 * rows * rows * k / base["seconds"] / 1e12
+        base["unit"] = "TFLOP/s"
+        line["cpu_baseline"] = base
+    return line
 
 
 def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
     """Device time per call of the other workloads (parity-test configurations, reported
     beside the headline): dense 4096x4096 row+column cast, the grouped MoE cast
-    (65536x7168, 64 token groups) and the 16x16 weight cast (28672x8192). Two input
-    copies rotate (the dense one fits L2: 8 copies rotate there)."""
+    (65536x7168, 64 token groups), the 16x16 weight cast (28672x8192) and the calibration
+    stream (200 activations of 8192x4096 through the fused cast and the decayed buffer at
+    decay 0.99; one step = one activation). Two input copies rotate (the dense one fits
+    L2: 8 copies rotate there; the stream's 200 activations are all distinct)."""
     import torch
 
     import precision_quantization_row_b200 as nv
@@ -524,6 +603,7 @@ def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
     torch.cuda.set_device(dist.local_rank)
     dev = torch.device("cuda", dist.local_rank)
     stream = torch.cuda.current_stream(dev)
+    offsets = None
     if config == "dense":
         x = inputs.dense().to(dev)
         m, k, g, copies = x.shape[0], x.shape[1], 1, 8
@@ -531,10 +611,16 @@ def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
         xh, offsets = inputs.moe()
         x = xh.to(dev)
         m, k, g, copies = x.shape[0], x.shape[1], len(offsets) - 1, 2
-    else:
+    elif config == "weight":
         x = inputs.weight().to(dev)
         m, k, g, copies = x.shape[0], x.shape[1], 1, 2
-    xs = [x] + [x.clone() for _ in range(copies - 1)]
+    else:   # calib
+        m, k, g, copies = 8192, 4096, 1, 200
+        x = None
+    if config == "calib":
+        xs = [inputs.calib_step(t, m, k, device=str(dev)) for t in range(copies)]
+    else:
+        xs = [x] + [x.clone() for _ in range(copies - 1)]
     ws = nv.new_workspace(m, k, g, device=dev)
     if config == "moe":
         outs = [None] * copies
@@ -544,12 +630,13 @@ def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
             outs[i % copies] = nv.quantize_grouped(xs[i % copies], offsets, absmax=bufs, decay=DECAY,
                                                    out=outs[i % copies], workspace=ws, stream=stream)
         byts = 2 * (2 * m * k) + 2 * (m * k // 2) + 2 * (m * k // 16) + 4 * m + 4 * g * k
-    elif config == "dense":
-        outs = [nv._outputs(m, k, nv.ROWWISE | nv.COLWISE, dev) for _ in range(copies)]
+    elif config in ("dense", "calib"):
+        nout = 2 if config == "calib" else copies
+        outs = [nv._outputs(m, k, nv.ROWWISE | nv.COLWISE, dev) for _ in range(nout)]
         buf = torch.zeros(1, dtype=torch.float32, device=dev)
 
         def step(i):
-            nv.quantize(xs[i % copies], absmax=buf, decay=DECAY, out=outs[i % copies], workspace=ws, stream=stream)
+            nv.quantize(xs[i % copies], absmax=buf, decay=DECAY, out=outs[i % nout], workspace=ws, stream=stream)
         byts = algo_bytes(m, k)
     else:
         outs = [None] * copies
@@ -558,21 +645,9 @@ def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
             outs[i % copies] = nv.quantize_weight_2d(xs[i % copies], out=outs[i % copies], workspace=ws,
                                                      stream=stream)
         byts = 2 * (2 * m * k) + m * k // 2 + m * k // 16 + 4 * m   # read twice, rowwise out
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def run():
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        ev1.record(stream)
-        ev1.synchronize()
-        return ev0.elapsed_time(ev1) / 1e3
-
-    with ClockSampler(dev.index) as clk:
-        secs = timed_region(dist, run, lambda: torch.cuda.synchronize(dev))
+    if config == "calib":
+        args.steps = copies   # one step per activation of the stream
+    secs, all_secs, clocks = timed_regions(args, dist, dev, stream, step)
     if nv.workspace_error(ws) != 0:
         raise RuntimeError("device error word set during the timed region")
     if dist.rank != 0:
@@ -580,36 +655,77 @@ def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
     peak, peak_kind = measured_peak()
     per = secs / args.steps
     achieved = byts / per / 1e9
-    return {
+    workload = {"dense": "dense_4096x4096_rowcol", "moe": "moe_grouped_65536x7168_g64_rowcol",
+                "weight": "weight_2d_28672x8192", "calib": "calibration_stream_200x8192x4096_decay0.99"}[config]
+    line = {
         "metric": "NVFP4 per-token cast: elems/s, achieved HBM GB/s, % of B200 HBM peak",
         "value": float(m) * k * args.steps * dist.world / secs, "unit": "elem/s", "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16->nvfp4", "data": "synthetic",
-        "config": {"workload": {"dense": "dense_4096x4096_rowcol", "moe": "moe_grouped_65536x7168_g64_rowcol",
-                                "weight": "weight_2d_28672x8192"}[config],
-                   "rows": m, "cols": k, "groups": g, "l2": f"{copies} rotating input copies"},
+        "config": {"workload": workload, "rows": m, "cols": k, "groups": g,
+                   "l2": f"{copies} rotating input copies" if config != "calib" else
+                         "200 distinct activations (the stream), 2 output sets"},
+        "timing": region_stats(all_secs),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_source": peak_kind, "algorithmic_bytes_per_call": byts},
-        "clocks": clk.summary(),
+                     "nominal_frac_8TBs": achieved / 8000.0, "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_call": byts},
+        "gpu_launches": nv.CAST_LAUNCHES * args.steps, "clocks": clocks,
     }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = config_oracle_baseline(config, xs, offsets, m, k)
+    return line
 
 
-def oracle_sample_rate(rows: int) -> tuple[float, str]:
-    """elems/s of the oracle's full row+col cast (with the absmax update) of the
-    first `rows` rows of the benchmark matrix, single-threaded."""
+def config_oracle_baseline(config: str, xs, offsets, m: int, k: int) -> dict:
+    """The oracle on a bounded sample of the workload, pinned to one core."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    if config == "calib":
+        # steps t = 0, 99 and 199 of the stream, each a full cast with the buffer update
+        ts = (0, 99, 199)
+        samples = [oracle._bits(xs[t].cpu()) for t in ts]
+
+        def run():
+            buf = 0.0
+            for s in samples:
+                buf = oracle.quantize(s, absmax=buf, decay=DECAY)["absmax"]
+        return oracle_baseline(len(ts) * m * k, run, "steps t = 0, 99, 199 of the stream (full casts and "
+                               "buffer updates); value = elem/s over the three")
+    if config == "moe":
+        # the first four token groups, one grouped cast
+        g4 = 4
+        rows = int(offsets[g4])
+        xb = oracle._bits(xs[0][:rows].cpu())
+        off = np.asarray(offsets[:g4 + 1], np.int64)
+        return oracle_baseline(rows * k, lambda: oracle.quantize_grouped(xb, off),
+                               f"the first {g4} token groups ({rows} rows) as one grouped cast")
+    if config == "weight":
+        rows = 2048
+        wb = oracle._bits(xs[0][:rows].cpu())
+        return oracle_baseline(rows * k, lambda: oracle.quantize_weight_2d(wb),
+                               f"rows 0..{rows - 1} of the weight (2D cast)")
+    xb = oracle._bits(xs[0].cpu())   # dense: the whole matrix
+    return oracle_baseline(m * k, lambda: oracle.quantize(xb, absmax=0.0, decay=DECAY),
+                           f"the whole {m}x{k} matrix, full row+col cast with the buffer update")
+
+
+def headline_oracle_baseline(rows: int) -> dict:
+    """The oracle's full row+col cast (with the absmax update) of the first `rows` rows of
+    the benchmark matrix, single-threaded and pinned to one core."""
     import oracle
     from precision_quantization_row_b200 import inputs
-    x = inputs.llm()[:rows].contiguous()
-    xb = oracle._bits(x)
-    t = time.perf_counter()
-    oracle.quantize(xb, absmax=0.0, decay=DECAY)
-    dt = time.perf_counter() - t
-    return rows * K / dt, f"rows 0..{rows - 1} of the {M}x{K} matrix ({rows * K} elements), full row+col cast"
+    oracle.build()
+    xb = oracle._bits(inputs.llm()[:rows].contiguous())
+    return oracle_baseline(rows * K, lambda: oracle.quantize(xb, absmax=0.0, decay=DECAY),
+                           f"rows 0..{rows - 1} of the {M}x{K} matrix ({rows * K} elements), full row+col cast")
 
 
 def run_reference(args, rank: int, world: int) -> dict | None:
-    """The oracle as it stands, single-threaded, on bounded row slices of the same
-    matrix; the slice is sized so that warm-up + timed steps take about two minutes."""
+    """The oracle as it stands, single-threaded and pinned to one core, on bounded row
+    slices of the same matrix; the slice is sized so that warm-up + timed steps take
+    about two minutes."""
     if rank != 0:
         return None
     import oracle
@@ -623,13 +739,20 @@ def run_reference(args, rank: int, world: int) -> dict | None:
     rows = int(120.0 / max(1, args.steps + args.warmup) / max(per_row, 1e-9)) // 16 * 16
     rows = max(16, min(1024, rows))
     samples = [oracle._bits(x[(i * rows) % M:(i * rows) % M + rows].contiguous()) for i in range(4)]
-    for i in range(args.warmup):
-        oracle.quantize(samples[i % 4], absmax=0.0, decay=DECAY)
-    t = time.perf_counter()
-    for i in range(args.steps):
-        oracle.quantize(samples[i % 4], absmax=0.0, decay=DECAY)
-    secs = time.perf_counter() - t
+
+    def run():
+        for i in range(args.warmup):
+            oracle.quantize(samples[i % 4], absmax=0.0, decay=DECAY)
+        t = time.perf_counter()
+        for i in range(args.steps):
+            oracle.quantize(samples[i % 4], absmax=0.0, decay=DECAY)
+        return time.perf_counter() - t
+
+    secs, _, core = pinned(run)
     value = rows * K * args.steps / secs
+    base = {"value": value, "unit": "elem/s", "cores": 1, "kind": "oracle", "pinned_core": core,
+            "sample": f"{rows}-row slices ({rows * K} elements) of the {M}x{K} matrix per step"}
+    base.update(cpu_info())
     return {
         "impl": "reference",
         "metric": "NVFP4 per-token cast: elems/s, achieved HBM GB/s, % of B200 HBM peak",
@@ -638,8 +761,7 @@ def run_reference(args, rank: int, world: int) -> dict | None:
         "vs_baseline": None, "dtype": "bf16->nvfp4 (e2m1 codes, e4m3 scales, fp32 amax)", "data": "synthetic",
         "config": {"workload": workload_name(M, K), "rows": M, "cols": K, "flags": "rowwise+columnwise",
                    "absmax_decay": DECAY, "parallelism": "single CPU thread"},
-        "cpu_baseline": {"value": value, "unit": "elem/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{rows}-row slices ({rows * K} elements) of the {M}x{K} matrix per step"},
+        "cpu_baseline": base,
         "e2e": {"value": value, "unit": "elem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -649,6 +771,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--repeats", type=int, default=0,
+                    help="timed regions of --steps steps (0: enough for about a second, 5..50)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--rows", type=int, default=16384, help="rows of the activation (profiling runs)")
     ap.add_argument("--cols", type=int, default=8192, help="columns of the activation (profiling runs)")
@@ -657,7 +781,7 @@ def main(argv=None):
     ap.add_argument("--op", choices=["cast", "dequant", "requant", "gemm"], default="cast",
                     help="cast: the per-token cast (the headline); dequant / requant / gemm: the secondary ops")
     ap.add_argument("--gemm-n", type=int, default=8192, help="N of --op gemm (M = --rows, K = --cols)")
-    ap.add_argument("--config", choices=["llm", "dense", "moe", "weight"], default="llm",
+    ap.add_argument("--config", choices=["llm", "dense", "moe", "weight", "calib"], default="llm",
                     help="llm: the headline activation; the others time the remaining workloads")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -668,28 +792,17 @@ def main(argv=None):
             print(json.dumps(line), flush=True)
         return
     dist = Dist(args.gpus)
-    if args.config != "llm":
-        try:
-            line = run_gpu_config(args, dist, args.config)
-            if line is not None:
-                print(json.dumps(line), flush=True)
-        finally:
-            dist.close()
-        return
-    if args.op != "cast":
-        try:
-            line = run_gpu_gemm(args, dist) if args.op == "gemm" else run_gpu_op(args, dist, args.op)
-            if line is not None:
-                print(json.dumps(line), flush=True)
-        finally:
-            dist.close()
-        return
     try:
-        line = run_gpu(args, dist)
-        if line is not None and dist.world == 1 and not args.no_cpu_baseline:
-            rate, sample = oracle_sample_rate(8192)
-            line["cpu_baseline"] = {"value": rate, "unit": "elem/s", "cores": 1, "kind": "oracle",
-                                    "sample": sample}
+        if args.config != "llm":
+            line = run_gpu_config(args, dist, args.config)
+        elif args.op == "gemm":
+            line = run_gpu_gemm(args, dist)
+        elif args.op != "cast":
+            line = run_gpu_op(args, dist, args.op)
+        else:
+            line = run_gpu(args, dist)
+            if line is not None and dist.world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = headline_oracle_baseline(8192)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

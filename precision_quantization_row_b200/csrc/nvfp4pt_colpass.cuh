@@ -3,15 +3,17 @@
 // group in amax_col. It reads x once more, straight into registers: no shared-memory
 // tiles of x, no block barriers in the loop.
 //
-// Layout of the work: a "task" is up to 256 rows x 32 columns of one token group,
-// given to one warp and taken in "steps" of 64 rows. In a step, lane l = 4q + s holds
-// the 16 rows 16s..16s+15 of the step's columns 4q..4q+3 (one 8-byte load per row),
-// encodes its four 16-row blocks and parks codes and scales in the warp's staging
-// area. After the task's last step the warp writes the task's columns: up to 128 code
-// bytes per column (one whole L2 line), eight lanes to a line so that each store
-// instruction covers four lines, and 16 scale bytes per column. Whole lines matter:
-// column outputs are strided by the group's row count, and lines written a sector at
-// a time, far apart in time, go back to DRAM a sector at a time.
+// Layout of the work: a "task" is up to 512 rows x 32 columns of one token group,
+// given to one warp and taken in "steps" of 64 rows. In a step, lane l = q + 8s holds
+// the 16 rows 16s..16s+15 of the step's columns 4q..4q+3 (one 8-byte load per row, so
+// eight consecutive lanes read one row's 64 bytes), encodes its four 16-row blocks and
+// parks codes and scales in the warp's staging area. After each 256 rows (a "half")
+// the warp writes their codes: up to 128 code bytes per column (one whole L2 line),
+// eight lanes to a line so that each store instruction covers four lines. After the
+// task's last step it writes 32 scale bytes per column (one whole 32-byte sector).
+// Whole lines and sectors matter: column outputs are strided by the group's row count,
+// and lines or sectors written in parts, far apart in time, go back to DRAM in parts
+// (a half-written sector costs a read of the sector before its write).
 //
 // Tasks are numbered row-task-major over all groups and walked backwards, each warp
 // prefetching the next step's rows into a second register buffer. With one token group the grid's warps take tasks
@@ -28,9 +30,10 @@ namespace nvfp4pt {
 constexpr int kColThreads = 512;   // one CTA per SM: 128 registers per thread
 constexpr int kColWarps = kColThreads / 32;
 constexpr int kStepRows = 64;      // rows of a step: four 16-row blocks
-constexpr int kTaskRows = 256;     // rows of a task: up to four steps
+constexpr int kTaskRows = 512;     // rows of a task: up to eight steps
+constexpr int kHalfRows = 256;     // rows whose codes are staged and written at once
 constexpr int kTaskCols = 32;      // columns of a task: 8 quads x 4
-constexpr int kColStageBytes = kTaskCols * (128 + 16);      // per warp: codes, scales
+constexpr int kColStageBytes = kTaskCols * (128 + 32);      // per warp: codes of a half, scales of a task
 constexpr int kSmemColPass = kColWarps * kColStageBytes;    // dynamic shared memory
 
 template <int MAXG>
@@ -83,7 +86,7 @@ struct ColTask {
     int32_t goff;
     int32_t grows;
     int32_t c0;
-    int32_t nrows;    // 16..256, a multiple of 16
+    int32_t nrows;    // 16..512, a multiple of 16
 };
 
 // Staging slot of 8-byte chunk k (16 rows) of column c: 16-byte chunk (k >> 1) ^ g(c)
@@ -112,7 +115,7 @@ __device__ __forceinline__ int group_of_task(const ColParams<MAXG>& p, int rt)
 template <int MAXG, bool NV = false>
 __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant__ ColParams<MAXG> p)
 {
-    // per warp: codes [column][16 chunks of 8 bytes] (swizzled), then scales [column][16]
+    // per warp: codes [column][16 chunks of 8 bytes] (swizzled), then scales [column][32]
     // The next cast's zeroing kernel may take its place early; it waits for this grid.
     griddep_launch_dependents();
     extern __shared__ __align__(16) uint8_t col_stage[];
@@ -122,8 +125,8 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int quad = lane >> 2;
-    const int blk = lane & 3;          // 16-row block of the step this lane loads
+    const int quad = lane & 7;         // columns 4 quad .. 4 quad + 3 of the task
+    const int blk = lane >> 3;         // 16-row block of the step this lane loads
     const int64_t cols = p.cols;
 
     // this warp's tasks: first, first - wstride, ... >= t0
@@ -201,16 +204,16 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
         return p.colmax ? __uint_as_float((uint32_t)p.colmax[i] << 16) : p.amax_col[i];
     };
     // With colmax, the fp32 amax_col output of (group, strip) comes from the warp that
-    // takes the group's first row task there: lane l holds column c0 + l's amax.
+    // takes the group's first row task there: lane l holds column c0 + 4 quad + blk's amax.
     auto publish_amax = [&](const ColTask& ct, float a) {
-        const int c = ct.c0 + lane;
+        const int c = ct.c0 + 4 * quad + blk;
         if (p.colmax && ct.row0 == ct.goff && c < cols) p.amax_col[(int64_t)g * cols + c] = a;
     };
     // outer scales of the quad's four columns: each lane finds one, the quad shares them
     auto outer_scales = [&](float a, float (&sc)[4]) {
         const float mine = s_enc_of(a);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) sc[j] = __shfl_sync(0xFFFFFFFFu, mine, (lane & ~3) | j);
+        for (int j = 0; j < 4; ++j) sc[j] = __shfl_sync(0xFFFFFFFFu, mine, (j << 3) | quad);
     };
 
     ColTask cur;
@@ -237,12 +240,12 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
 
     uint8_t* xc = col_stage + warp * kColStageBytes;
     uint8_t* xs = xc + kTaskCols * 128;
-    // This lane's slots: column 4q+j, block kb = 4*step + blk goes to
-    // stage_off(4q+j, kb) = xq + 128j + 16*(hg ^ j), hg = (kb >> 1) ^ G(q), where
-    // g(4q+j) = j ^ G(q) with G(q) = 4(q & 1) ^ (q & 6); its scale byte to
-    // xsq + 16j + 4*step.
+    // This lane's slots: column 4q+j, block kb = 4*(step & 3) + blk of the current half
+    // goes to stage_off(4q+j, kb) = xq + 128j + 16*(hg ^ j), hg = (kb >> 1) ^ G(q), where
+    // g(4q+j) = j ^ G(q) with G(q) = 4(q & 1) ^ (q & 6); its scale byte (block
+    // 4*step + blk of the task) to xsq + 32j + 4*step.
     uint8_t* xq = xc + 512 * quad + 8 * (blk & 1);
-    uint8_t* xsq = xs + 64 * quad + blk;
+    uint8_t* xsq = xs + 128 * quad + blk;
     const int gq = (4 * (quad & 1)) ^ (quad & 6);
     const uint64_t pol_out = l2_evict_first();
     float sc[4];
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
         block_pair_scales_x2(bf16_lo(m[1]), bf16_hi(m[1]), sc[2], sc[3], sf23, e[2], e[3], rcp_tab);
 
         // codes and scales of this lane's block of each column -> staging
-        const int hg = (2 * step + (blk >> 1)) ^ gq;
+        const int hg = (2 * (step & 3) + (blk >> 1)) ^ gq;
         uint8_t* xsb = xsq + 4 * step;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -315,14 +318,15 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
             const uint32_t lo = (j & 1) ? encode8_strided<true>(v, 0, w, e[j]) : encode8_strided<false>(v, 0, w, e[j]);
             const uint32_t hi = (j & 1) ? encode8_strided<true>(v, 8, w, e[j]) : encode8_strided<false>(v, 8, w, e[j]);
             *reinterpret_cast<uint2*>(xq + 128 * j + 16 * (hg ^ j)) = make_uint2(lo, hi);
-            xsb[16 * j] = (uint8_t)(((j < 2) ? sf01 : sf23) >> (8 * (j & 1)));
+            xsb[32 * j] = (uint8_t)(((j < 2) ? sf01 : sf23) >> (8 * (j & 1)));
         }
 
-        if (step == 0) {
-            // task done: write the task's columns out of staging
+        if ((step & 3) == 0) {
+            // a half done: write its codes out of staging (the half's rows start at
+            // 64 * step of the task)
             __syncwarp();
-            const int nblk = cur.nrows / 16;
-            const int lrow = cur.row0 - cur.goff;
+            const int nblk = min(16, cur.nrows / 16 - 4 * step);
+            const int lrow = cur.row0 - cur.goff + kStepRows * step;
             const int64_t gq = cols * cur.goff / 2 + lrow / 2;    // column 0's code bytes, then
             const int64_t cstride = cur.grows / 2;                //   one column every cstride
             const bool wide = p.q_col_32 && (cur.grows & 63) == 0;
@@ -339,28 +343,39 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
                         stg16_ef(p.q_col + gq + (int64_t)c * cstride + 16 * k, a, pol_out);
                     }
                 }
-            }
-            // lane j: column j's scales (and its codes when not aligned for the above)
-            const int c = cur.c0 + lane;
-            if (c < cols) {
-                uint8_t* q = p.q_col + gq + (int64_t)c * cstride;
-                uint8_t* sf = p.sf_col + cols * cur.goff / 16 + (int64_t)c * (cur.grows / 16) + lrow / 16;
-                if (!wide) {
+            } else if (cur.c0 + lane < cols) {
+                // lane j: column j's codes
+                uint8_t* q = p.q_col + gq + (int64_t)(cur.c0 + lane) * cstride;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        if (i < nblk) {
-                            const uint2 a = *reinterpret_cast<const uint2*>(xc + stage_off(lane, i));
-                            stg8_ef(q + 8 * i, a.x, a.y, pol_out);
-                        }
+                for (int i = 0; i < 16; ++i) {
+                    if (i < nblk) {
+                        const uint2 a = *reinterpret_cast<const uint2*>(xc + stage_off(lane, i));
+                        stg8_ef(q + 8 * i, a.x, a.y, pol_out);
                     }
                 }
-                const uint4 s16 = *reinterpret_cast<const uint4*>(xs + 16 * lane);
-                if (nblk == 16 && (reinterpret_cast<uintptr_t>(sf) & 15u) == 0) {
-                    stg16_ef(sf, s16, pol_out);
+            }
+            __syncwarp();   // staging is written again by the next step
+        }
+        if (step == 0) {
+            // task done: lane j writes column j's block scales, one whole 32-byte sector
+            // per column when the task has 512 rows
+            const int nblk = cur.nrows / 16;
+            const int lrow = cur.row0 - cur.goff;
+            const int c = cur.c0 + lane;
+            if (c < cols) {
+                uint8_t* sf = p.sf_col + cols * cur.goff / 16 + (int64_t)c * (cur.grows / 16) + lrow / 16;
+                const uint4 s0 = *reinterpret_cast<const uint4*>(xs + 32 * lane);
+                const uint4 s1 = *reinterpret_cast<const uint4*>(xs + 32 * lane + 16);
+                const uintptr_t al = reinterpret_cast<uintptr_t>(sf);
+                if (nblk == 32 && (al & 31u) == 0) {
+                    stg32_ef(sf, s0, s1, pol_out);
+                } else if (nblk == 32 && (al & 15u) == 0) {
+                    stg16_ef(sf, s0, pol_out);
+                    stg16_ef(sf + 16, s1, pol_out);
                 } else {
-                    const uint32_t sw[4] = {s16.x, s16.y, s16.z, s16.w};
+                    const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < 8; ++i)
                         if (4 * i < nblk) stg_bytes(sf + 4 * i, sw[i], min(4, nblk - 4 * i));
                 }
             }

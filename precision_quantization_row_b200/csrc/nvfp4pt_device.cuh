@@ -448,6 +448,12 @@ __device__ __forceinline__ void stg16_ef(uint8_t* p, uint4 v, uint64_t pol)   //
     asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;"
                  :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol) : "memory");
 }
+__device__ __forceinline__ void stg32_ef(uint8_t* p, uint4 a, uint4 b, uint64_t pol)   // 32-byte aligned
+{
+    asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;"
+                 :: "l"(p), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "l"(pol)
+                 : "memory");
+}
 __device__ __forceinline__ void stg8_ef(uint8_t* p, uint32_t a, uint32_t b, uint64_t pol)   // 8-byte aligned
 {
     asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" :: "l"(p), "r"(a), "r"(b), "l"(pol) : "memory");
