@@ -74,6 +74,14 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_dequantize_rows.restype = ctypes.c_int
         _lib.oracle_gemm_per_token.argtypes = [P, P, P, I64, P, P, P, I64, I64, P, P]
         _lib.oracle_gemm_per_token.restype = ctypes.c_int
+        U32, U64 = ctypes.c_uint32, ctypes.c_uint64
+        _lib.oracle_philox4x32_10.argtypes, _lib.oracle_philox4x32_10.restype = [P, P, P], None
+        _lib.oracle_sr_word.argtypes, _lib.oracle_sr_word.restype = [I64, I64, U64, U64], U32
+        _lib.oracle_rht16.argtypes, _lib.oracle_rht16.restype = [P, U32, P], None
+        _lib.oracle_e2m1_sr.argtypes, _lib.oracle_e2m1_sr.restype = [F, U32], U8
+        _lib.oracle_quantize_colwise_opts.argtypes = [P, I64, I64, P, ctypes.c_int, ctypes.c_int, U32,
+                                                      ctypes.c_int, U64, U64, P, P, P]
+        _lib.oracle_quantize_colwise_opts.restype = ctypes.c_int
     return _lib
 
 
@@ -314,3 +322,53 @@ def gemm_per_token(qa, sfa, amax_a, qb, sfb, amax_b):
     if st == -2:
         raise ValueError("oracle_gemm_per_token: a block scale is not a non-negative finite e4m3fn code")
     return out, mag
+
+
+# ------------------------------------------- columnwise options: RHT and SR
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    """oracle_philox4x32_10: four 32-bit words of Philox4x32-10 at counter ctr (4 words)
+    with key (2 words)."""
+    c = np.ascontiguousarray(np.asarray(ctr, np.uint32))
+    k = np.ascontiguousarray(np.asarray(key, np.uint32))
+    out = np.zeros(4, np.uint32)
+    lib().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def sr_word(m: int, k: int, seed: int, offset: int) -> int:
+    """The random word of columnwise element (row m, column k)."""
+    return int(lib().oracle_sr_word(m, k, seed, offset))
+
+
+def rht16(v, signs: int) -> np.ndarray:
+    """(1/4) H16 S v by the four binary32 butterfly stages."""
+    a = np.ascontiguousarray(np.asarray(v, np.float32).reshape(16))
+    out = np.zeros(16, np.float32)
+    lib().oracle_rht16(_ptr(a), signs, _ptr(out))
+    return out
+
+
+def e2m1_sr(y: float, r: int) -> int:
+    return int(lib().oracle_e2m1_sr(y, r))
+
+
+def quantize_colwise_opts(x, offsets=None, rht: bool = False, rht_signs: int = 0, sr: bool = False,
+                          seed: int = 0, offset: int = 0) -> dict:
+    """The columnwise direction with the RHT / SR options. offsets None: one group, and
+    the outputs are shaped as quantize's ([K, M/2], [K, M/16], [K]); else as
+    quantize_grouped's (flat codes and scales, amax_col [G, K])."""
+    xb = _bits(x)
+    M, K = xb.shape
+    off = np.ascontiguousarray(np.asarray([0, M] if offsets is None else offsets, np.int64))
+    G = off.size - 1
+    q = np.zeros(K * M // 2, np.uint8)
+    sf = np.zeros(K * M // 16, np.uint8)
+    am = np.zeros((G, K), np.float32)
+    rc = lib().oracle_quantize_colwise_opts(_ptr(xb), M, K, _ptr(off), G, int(rht), rht_signs & 0xFFFF, int(sr),
+                                            seed, offset, _ptr(q), _ptr(sf), _ptr(am))
+    if rc != 0:
+        raise ValueError("oracle_quantize_colwise_opts: bad shape or offsets")
+    if offsets is None:
+        return {"q_col": q.reshape(K, M // 2), "sf_col": sf.reshape(K, M // 16), "amax_col": am.reshape(K)}
+    return {"q_col": q, "sf_col": sf, "amax_col": am}

@@ -481,3 +481,145 @@ void oracle_f32_to_bf16_array(const float* v, int64_t n, uint16_t* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f32_to_bf16(v[i]);
 }
+
+/* ------------------------------------- columnwise options: RHT and SR */
+
+/* TransformerEngine PR #3045, Changes: an opt-in random Hadamard transform (RHT) and
+ * opt-in stochastic rounding (SR) on the per-token path, off by default; its review:
+ * the row direction never uses RHT. The pages fix neither the transform size, the
+ * signs, the evaluation order nor the random numbers. The readings taken (each listed
+ * in the design notes):
+ *  - RHT acts on each columnwise 16-element block (16 consecutive rows of one column
+ *    inside a token group): v' = (1/4) H16 S v, H16 the Sylvester Hadamard matrix
+ *    (H[i][j] = (-1)^popcount(i & j)), S = diag(s_j), s_j = -1 where bit j of a
+ *    caller-given 16-bit mask is set. Orthogonal: (1/4 H16)^2 = I. Evaluated as the
+ *    radix-2 butterfly in four stages (pairs i, i+h for h = 1, 2, 4, 8: sum and
+ *    difference, each one binary32 rounding), then the exact multiply by 1/4.
+ *  - The columnwise cast then runs on v' exactly as on x: the column amax is the
+ *    max |v'| over the group's rows, and the block steps are unchanged.
+ *  - SR replaces the final E2M1 rounding: with a = |y| < 6, lo <= a < hi the
+ *    neighbouring E2M1 values and f = (a - lo) / (hi - lo) (exact), a 32-bit random
+ *    word r rounds up iff r < ceil(f * 2^32), so up with probability f up to 2^-32;
+ *    a >= 6 saturates to 6; the sign bit is y's.
+ *  - The random word of columnwise element (row m, column k) is output m % 4 of
+ *    Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) with counter
+ *    (m / 4, k, lo32(offset), hi32(offset)) and key (lo32(seed), hi32(seed)). */
+
+/* Philox4x32 with 10 rounds: each round maps the counter (c0, c1, c2, c3) with the key
+ * (k0, k1) to (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)) with the
+ * multipliers M0 = 0xD2511F53, M1 = 0xCD9E8D57; between rounds the key grows by the
+ * Weyl constants (0x9E3779B9, 0xBB67AE85). */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n1 = (uint32_t)p1;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        const uint32_t n3 = (uint32_t)p0;
+        c0 = n0;
+        c1 = n1;
+        c2 = n2;
+        c3 = n3;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+/* The random word of columnwise element (row m, column k). */
+uint32_t oracle_sr_word(int64_t m, int64_t k, uint64_t seed, uint64_t offset)
+{
+    const uint32_t ctr[4] = {(uint32_t)(m >> 2), (uint32_t)k, (uint32_t)offset, (uint32_t)(offset >> 32)};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    oracle_philox4x32_10(ctr, key, out);
+    return out[m & 3];
+}
+
+/* v' = (1/4) H16 S v by the four butterfly stages (see above). */
+void oracle_rht16(const float* v, uint32_t signs, float* out)
+{
+    float w[16];
+    for (int j = 0; j < 16; ++j) w[j] = ((signs >> j) & 1u) ? -v[j] : v[j];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int i = 0; i < 16; ++i)
+            if ((i & h) == 0) {
+                const float a = w[i], b = w[i + h];
+                w[i] = a + b;
+                w[i + h] = a - b;
+            }
+    for (int j = 0; j < 16; ++j) out[j] = w[j] * 0.25f;
+}
+
+/* Stochastic rounding of y to E2M1 with the random word r (see above). */
+uint8_t oracle_e2m1_sr(float y, uint32_t r)
+{
+    const uint8_t sign = signbit(y) ? 0x8 : 0x0;
+    const double a = fabs((double)y);
+    if (a >= 6.0) return sign | 0x7;
+    int c = 0;
+    while (c < 7 && kE2M1[c + 1] <= a) ++c;
+    const double f = (a - kE2M1[c]) / (kE2M1[c + 1] - kE2M1[c]);   /* exact */
+    const uint64_t t = (uint64_t)ceil(ldexp(f, 32));
+    return sign | (uint8_t)((uint64_t)r < t ? c + 1 : c);
+}
+
+/* The columnwise direction of the grouped cast with the options: rht (0/1) with the
+ * sign mask, sr (0/1) with seed and offset. Outputs and layouts as in
+ * oracle_quantize_grouped (amax_col [G, K] of the transformed values when rht).
+ * Returns 0, or -1 on bad shape/offsets. */
+int oracle_quantize_colwise_opts(const uint16_t* x, int64_t M, int64_t K, const int64_t* offsets, int G,
+                                 int rht, uint32_t rht_signs, int sr, uint64_t seed, uint64_t offset,
+                                 uint8_t* q_col, uint8_t* sf_col, float* amax_col)
+{
+    if (!shape_ok(M, K) || G < 1) return -1;
+    if (offsets[0] != 0 || offsets[G] != M) return -1;
+    for (int g = 0; g < G; ++g)
+        if (offsets[g + 1] < offsets[g] || offsets[g] % 16 != 0) return -1;
+    float v[16], y[16];
+    for (int g = 0; g < G; ++g) {
+        const int64_t r0 = offsets[g], m = offsets[g + 1] - offsets[g];
+        uint8_t* qg = q_col + K * r0 / 2;
+        uint8_t* sg = sf_col + K * r0 / 16;
+        for (int64_t c = 0; c < K; ++c) {
+            /* the column's amax over the group, of the (transformed) values */
+            float amax = 0.0f;
+            for (int64_t b = 0; b < m / 16; ++b) {
+                for (int i = 0; i < 16; ++i) v[i] = oracle_bf16_to_f32(x[(r0 + 16 * b + i) * K + c]);
+                if (rht) oracle_rht16(v, rht_signs, v);
+                for (int i = 0; i < 16; ++i)
+                    if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+            }
+            amax_col[(int64_t)g * K + c] = amax;
+            const float s_enc = oracle_s_enc(amax);
+            for (int64_t b = 0; b < m / 16; ++b) {
+                for (int i = 0; i < 16; ++i) v[i] = oracle_bf16_to_f32(x[(r0 + 16 * b + i) * K + c]);
+                if (rht) oracle_rht16(v, rht_signs, v);
+                float ba = 0.0f;
+                for (int i = 0; i < 16; ++i)
+                    if (fabsf(v[i]) > ba) ba = fabsf(v[i]);
+                const uint8_t sf = oracle_e4m3(oracle_block_scale_arg(ba, s_enc));
+                const float enc = oracle_block_enc(sf, s_enc);
+                uint8_t codes[16];
+                for (int i = 0; i < 16; ++i) {
+                    y[i] = v[i] * enc;
+                    codes[i] = sr ? oracle_e2m1_sr(y[i], oracle_sr_word(r0 + 16 * b + i, c, seed, offset))
+                                  : oracle_e2m1(y[i]);
+                }
+                for (int j = 0; j < 8; ++j)
+                    qg[c * (m / 2) + 8 * b + j] = (uint8_t)(codes[2 * j] | (codes[2 * j + 1] << 4));
+                sg[c * (m / 16) + b] = sf;
+            }
+        }
+    }
+    return 0;
+}
