@@ -694,21 +694,26 @@ def config_oracle_baseline(config: str, xs, offsets, m: int, k: int) -> dict:
         return oracle_baseline(len(ts) * m * k, run, "steps t = 0, 99, 199 of the stream (full casts and "
                                "buffer updates); value = elem/s over the three")
     if config == "moe":
-        # the first four token groups, one grouped cast
-        g4 = 4
+        # the first sixteen token groups, one grouped cast (about 10 s of one core)
+        g4 = 16
         rows = int(offsets[g4])
         xb = oracle._bits(xs[0][:rows].cpu())
         off = np.asarray(offsets[:g4 + 1], np.int64)
         return oracle_baseline(rows * k, lambda: oracle.quantize_grouped(xb, off),
                                f"the first {g4} token groups ({rows} rows) as one grouped cast")
     if config == "weight":
-        rows = 2048
+        rows = 28672   # the whole weight (about 7 s of one core)
         wb = oracle._bits(xs[0][:rows].cpu())
         return oracle_baseline(rows * k, lambda: oracle.quantize_weight_2d(wb),
                                f"rows 0..{rows - 1} of the weight (2D cast)")
-    xb = oracle._bits(xs[0].cpu())   # dense: the whole matrix
-    return oracle_baseline(m * k, lambda: oracle.quantize(xb, absmax=0.0, decay=DECAY),
-                           f"the whole {m}x{k} matrix, full row+col cast with the buffer update")
+    xb = oracle._bits(xs[0].cpu())   # dense: the whole matrix, five times (about 10 s of one core)
+
+    def run_dense():
+        buf = 0.0
+        for _ in range(5):
+            buf = oracle.quantize(xb, absmax=buf, decay=DECAY)["absmax"]
+    return oracle_baseline(5 * m * k, run_dense,
+                           f"the whole {m}x{k} matrix five times, full row+col cast with the buffer update")
 
 
 def headline_oracle_baseline(rows: int) -> dict:
@@ -802,7 +807,7 @@ def main(argv=None):
         else:
             line = run_gpu(args, dist)
             if line is not None and dist.world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = headline_oracle_baseline(8192)
+                line["cpu_baseline"] = headline_oracle_baseline(12288)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

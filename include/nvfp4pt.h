@@ -134,6 +134,53 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_grouped(const void* x_bf16, int64_t 
                                         void* workspace, cudaStream_t stream);
 
 /*
+ * Columnwise options of nvfp4pt_quantize_grouped_opts (TransformerEngine PR #3045,
+ * Changes: opt-in RHT / SR on the per-token path, off by default; its review: the row
+ * direction never uses RHT). The pages fix neither the transform nor the random
+ * numbers; the readings taken:
+ *   NVFP4PT_COL_RHT  each columnwise 16-element block v (16 consecutive rows of a column
+ *                    inside a token group) is replaced by v' = (1/4) H16 S v before the
+ *                    columnwise cast: H16 the Sylvester Hadamard matrix (entry (i, j) =
+ *                    (-1)^popcount(i & j)), S the diagonal of signs with -1 where bit j of
+ *                    rht_signs is set. It is evaluated as four radix-2 butterfly stages
+ *                    (pairs i, i + h, h = 1, 2, 4, 8: sum and difference, one binary32
+ *                    rounding each), then the exact multiply by 1/4. amax_col is then
+ *                    max |v'| over the group's rows; the block steps are unchanged.
+ *   NVFP4PT_COL_SR   the columnwise E2M1 rounding of y = RN(v * enc) is stochastic: with
+ *                    a = |y| < 6 between the E2M1 neighbours lo <= a < hi and the exact
+ *                    fraction f = (a - lo) / (hi - lo), the random word r rounds up iff
+ *                    r < ceil(f * 2^32); a >= 6 gives 6; the sign is y's. The word of
+ *                    element (row m, column k) is output m % 4 of Philox4x32-10 (Salmon
+ *                    et al., SC'11) at counter (m / 4, k, lo32(sr_offset), hi32(sr_offset))
+ *                    with key (lo32(sr_seed), hi32(sr_seed)).
+ * The rowwise direction and the running buffers are those of the call without options.
+ */
+enum { NVFP4PT_COL_RHT = 1, NVFP4PT_COL_SR = 2 };
+typedef struct nvfp4pt_colwise_options {
+    int flags;              /* NVFP4PT_COL_RHT and/or NVFP4PT_COL_SR; 0: none     */
+    uint32_t rht_signs;     /* bits 0..15: the sign mask S                        */
+    uint64_t sr_seed;       /* Philox key                                         */
+    uint64_t sr_offset;     /* Philox counter words 2-3 (e.g. the training step)  */
+} nvfp4pt_colwise_options;
+
+/*
+ * nvfp4pt_quantize_grouped_opts -- nvfp4pt_quantize_grouped with columnwise options
+ * (NULL or flags 0: exactly nvfp4pt_quantize_grouped). One token group (offsets {0,
+ * rows}) gives the ungrouped cast's outputs. With options the columnwise direction
+ * needs rows of at most 16384 elements (cols <= 16384), else NVFP4PT_ERR_SHAPE; flags
+ * outside NVFP4PT_COL_RHT | NVFP4PT_COL_SR give NVFP4PT_ERR_FLAGS. Workspace as in
+ * nvfp4pt_quantize_grouped. With NVFP4PT_COL_RHT the call launches one more kernel
+ * (the sweep that finds the column amax of the transformed values).
+ */
+NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_grouped_opts(const void* x_bf16, int64_t rows, int64_t cols,
+                                                         const int64_t* offsets_host, int num_groups, int flags,
+                                                         uint8_t* q_row, uint8_t* sf_row, float* amax_row,
+                                                         uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                                         float* absmax_bufs, float decay,
+                                                         const nvfp4pt_colwise_options* opts, void* workspace,
+                                                         cudaStream_t stream);
+
+/*
  * nvfp4pt_quantize_weight_2d -- the opt-in 2D weight cast (PR #3045, Changes:
  * "transposition-invariant 16x16 cast emitted in per-token layout").
  * Each row keeps its own s_enc from amax_row; the 16 rows of a band share one E4M3

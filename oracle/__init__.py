@@ -79,7 +79,7 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_sr_word.argtypes, _lib.oracle_sr_word.restype = [I64, I64, U64, U64], U32
         _lib.oracle_rht16.argtypes, _lib.oracle_rht16.restype = [P, U32, P], None
         _lib.oracle_e2m1_sr.argtypes, _lib.oracle_e2m1_sr.restype = [F, U32], U8
-        _lib.oracle_quantize_colwise_opts.argtypes = [P, I64, I64, P, ctypes.c_int, ctypes.c_int, U32,
+        _lib.oracle_quantize_colwise_opts.argtypes = [P, I64, I64, I64, P, ctypes.c_int, ctypes.c_int, U32,
                                                       ctypes.c_int, U64, U64, P, P, P]
         _lib.oracle_quantize_colwise_opts.restype = ctypes.c_int
     return _lib
@@ -354,10 +354,11 @@ def e2m1_sr(y: float, r: int) -> int:
 
 
 def quantize_colwise_opts(x, offsets=None, rht: bool = False, rht_signs: int = 0, sr: bool = False,
-                          seed: int = 0, offset: int = 0) -> dict:
+                          seed: int = 0, offset: int = 0, col_base: int = 0) -> dict:
     """The columnwise direction with the RHT / SR options. offsets None: one group, and
     the outputs are shaped as quantize's ([K, M/2], [K, M/16], [K]); else as
-    quantize_grouped's (flat codes and scales, amax_col [G, K])."""
+    quantize_grouped's (flat codes and scales, amax_col [G, K]). col_base: the column
+    index of x's first column in the full matrix (for the random words)."""
     xb = _bits(x)
     M, K = xb.shape
     off = np.ascontiguousarray(np.asarray([0, M] if offsets is None else offsets, np.int64))
@@ -365,7 +366,8 @@ def quantize_colwise_opts(x, offsets=None, rht: bool = False, rht_signs: int = 0
     q = np.zeros(K * M // 2, np.uint8)
     sf = np.zeros(K * M // 16, np.uint8)
     am = np.zeros((G, K), np.float32)
-    rc = lib().oracle_quantize_colwise_opts(_ptr(xb), M, K, _ptr(off), G, int(rht), rht_signs & 0xFFFF, int(sr),
+    rc = lib().oracle_quantize_colwise_opts(_ptr(xb), M, K, col_base, _ptr(off), G, int(rht), rht_signs & 0xFFFF,
+                                            int(sr),
                                             seed, offset, _ptr(q), _ptr(sf), _ptr(am))
     if rc != 0:
         raise ValueError("oracle_quantize_colwise_opts: bad shape or offsets")

@@ -576,9 +576,10 @@ uint8_t oracle_e2m1_sr(float y, uint32_t r)
 /* The columnwise direction of the grouped cast with the options: rht (0/1) with the
  * sign mask, sr (0/1) with seed and offset. Outputs and layouts as in
  * oracle_quantize_grouped (amax_col [G, K] of the transformed values when rht).
- * Returns 0, or -1 on bad shape/offsets. */
-int oracle_quantize_colwise_opts(const uint16_t* x, int64_t M, int64_t K, const int64_t* offsets, int G,
-                                 int rht, uint32_t rht_signs, int sr, uint64_t seed, uint64_t offset,
+ * col_base: the index of x's first column in the full matrix (x may be a column
+ * slice of it), which the random words use. Returns 0, or -1 on bad shape/offsets. */
+int oracle_quantize_colwise_opts(const uint16_t* x, int64_t M, int64_t K, int64_t col_base, const int64_t* offsets,
+                                 int G, int rht, uint32_t rht_signs, int sr, uint64_t seed, uint64_t offset,
                                  uint8_t* q_col, uint8_t* sf_col, float* amax_col)
 {
     if (!shape_ok(M, K) || G < 1) return -1;
@@ -612,7 +613,7 @@ int oracle_quantize_colwise_opts(const uint16_t* x, int64_t M, int64_t K, const 
                 uint8_t codes[16];
                 for (int i = 0; i < 16; ++i) {
                     y[i] = v[i] * enc;
-                    codes[i] = sr ? oracle_e2m1_sr(y[i], oracle_sr_word(r0 + 16 * b + i, c, seed, offset))
+                    codes[i] = sr ? oracle_e2m1_sr(y[i], oracle_sr_word(r0 + 16 * b + i, col_base + c, seed, offset))
                                   : oracle_e2m1(y[i]);
                 }
                 for (int j = 0; j < 8; ++j)

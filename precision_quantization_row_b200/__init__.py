@@ -37,7 +37,17 @@ EXPORTS = (
     "nvfp4pt_quantize_weight_2d", "nvfp4pt_update_absmax", "nvfp4pt_workspace_error",
     "nvfp4pt_quantize_grouped_noalloc", "nvfp4pt_quantize_timed", "nvfp4pt_dequantize", "nvfp4pt_requantize_workspace_bytes",
     "nvfp4pt_requantize_colwise", "nvfp4pt_gemm_workspace_bytes", "nvfp4pt_gemm_per_token",
+    "nvfp4pt_quantize_grouped_opts",
 )
+
+COL_RHT = 1   # NVFP4PT_COL_RHT
+COL_SR = 2    # NVFP4PT_COL_SR
+
+
+class ColwiseOptions(ctypes.Structure):
+    """nvfp4pt_colwise_options."""
+    _fields_ = [("flags", ctypes.c_int), ("rht_signs", ctypes.c_uint32), ("sr_seed", ctypes.c_uint64),
+                ("sr_offset", ctypes.c_uint64)]
 
 
 class Nvfp4ptError(RuntimeError):
@@ -70,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_dequantize.argtypes = [P, P, P, I64, I64, P, P]
         L.nvfp4pt_requantize_workspace_bytes.argtypes = [I64, I64, I]
         L.nvfp4pt_requantize_colwise.argtypes = [P, P, P, I64, I64, P, I, P, P, P, P, F, P, P]
+        L.nvfp4pt_quantize_grouped_opts.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, F, P, P, P]
         L.nvfp4pt_gemm_workspace_bytes.argtypes = []
         L.nvfp4pt_gemm_per_token.argtypes = [P, P, P, I64, P, P, P, I64, I64, P, P, P]
         for name in EXPORTS[2:]:
@@ -336,6 +347,37 @@ def quantize_grouped(x: torch.Tensor, offsets, flags: int = ROWWISE | COLWISE, a
     st = lib().nvfp4pt_quantize_grouped(_ptr(x), rows, cols, off, G, flags, *p, pa, ctypes.c_float(decay), pw,
                                         _stream(stream, x.device))
     _check("nvfp4pt_quantize_grouped", st)
+    return out
+
+
+def quantize_grouped_opts(x: torch.Tensor, offsets=None, flags: int = ROWWISE | COLWISE,
+                          absmax: torch.Tensor | None = None, decay: float = 0.0, rht: bool = False,
+                          rht_signs: int = 0, sr: bool = False, seed: int = 0, offset: int = 0,
+                          out: dict | None = None, workspace: torch.Tensor | None = None,
+                          stream: torch.cuda.Stream | None = None) -> dict:
+    """nvfp4pt_quantize_grouped_opts: the cast with the columnwise options (the Hadamard
+    transform of each columnwise 16-row block with the sign mask rht_signs; stochastic
+    rounding with the Philox seed and offset). offsets None: one group, and the outputs
+    are shaped as quantize's."""
+    _require_2d(x, "x", torch.bfloat16)
+    rows, cols = x.shape
+    dev = x.get_device()
+    offs = [0, rows] if offsets is None else list(offsets)
+    off = (ctypes.c_int64 * len(offs))(*[int(o) for o in offs])
+    G = len(offs) - 1
+    if out is None:
+        out = _outputs(rows, cols, flags, x.device) if offsets is None else \
+            _outputs(rows, cols, flags, x.device, col_rows=rows, groups=G)
+    ws = new_workspace(rows, cols, max(G, 1), x.device) if workspace is None else workspace
+    p = _out_ptrs(out, flags, rows, cols, max(G, 1), dev)
+    pa = _opt_buf(absmax, "absmax", torch.float32, max(G, 1), dev)
+    pw = _buf(ws, "workspace", torch.uint8, workspace_bytes(rows, cols, max(G, 1)), dev)
+    _require_cuda(x, "x")
+    opts = ColwiseOptions((COL_RHT if rht else 0) | (COL_SR if sr else 0), rht_signs & 0xFFFF,
+                          seed & (2**64 - 1), offset & (2**64 - 1))
+    st = lib().nvfp4pt_quantize_grouped_opts(_ptr(x), rows, cols, off, G, flags, *p, pa, ctypes.c_float(decay),
+                                             ctypes.byref(opts), pw, _stream(stream, x.device))
+    _check("nvfp4pt_quantize_grouped_opts", st)
     return out
 
 

@@ -60,7 +60,9 @@ nvfp4pt_status device_state(DeviceState** out)
                     return NVFP4PT_ERR_CUDA;
             }
             const void* colpasses[] = {(const void*)colpass<1, false>, (const void*)colpass<kMaxGroups, false>,
-                                       (const void*)colpass<1, true>, (const void*)colpass<kMaxGroups, true>};
+                                       (const void*)colpass<1, true>, (const void*)colpass<kMaxGroups, true>,
+                                       (const void*)colpass<1, false, kColOpts>,
+                                       (const void*)colpass<kMaxGroups, false, kColOpts>};
             for (const void* f : colpasses) {
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColPass) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
@@ -191,6 +193,15 @@ cudaError_t launch_rowpass(const RowShape& rs, const RowParams<MAXG>& rp, cudaSt
     return launch(rowpass<MAXG, 1, 1, NV>, grid, 0, stream, rp, true, kRowThreads);
 }
 
+// The columnwise options of a call (nvfp4pt_colwise_options), as the kernels take them.
+struct ColOptions {
+    bool rht;
+    uint32_t rht_signs;
+    bool sr;
+    uint64_t seed;
+    uint64_t offset;
+};
+
 // NVFP4 rowwise data as the cast's source (the requantization): codes, scales, row
 // amaxes, and room for the rows' decode scales.
 struct NvSource {
@@ -204,7 +215,8 @@ template <int MAXG>
 nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t* off, int G, int flags,
                         uint8_t* q_row, uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col,
                         float* amax_col, float* absmax, float decay, bool w2d, void* ws, cudaStream_t stream,
-                        void* const* events = nullptr, bool full_ws = true, const NvSource* nv = nullptr)
+                        void* const* events = nullptr, bool full_ws = true, const NvSource* nv = nullptr,
+                        const ColOptions* co = nullptr)
 {
     // events[0] before the first launch, events[i] after the i-th (measurement hook)
     auto mark = [&](int i) -> bool {
@@ -219,7 +231,11 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
     // The 1D cast of rows up to kRowPassMaxCols wide encodes rows in the amax pass.
     const bool row_pass = !w2d && cols <= kRowPassMaxCols;
     // bf16 column maxima in the workspace (8 columns per atomic), else fp32 atomics
-    uint16_t* colmax = (row_pass && do_col && full_ws) ? ws_colmax(ws, G) : nullptr;
+    // With the transform the column amax is of the transformed values: a sweep of its
+    // own accumulates it in amax_col, and the row pass takes no column maxima.
+    const bool opts = do_col && co && (co->rht || co->sr);
+    const bool xf_amax = opts && co->rht;
+    uint16_t* colmax = (row_pass && do_col && full_ws && !xf_amax) ? ws_colmax(ws, G) : nullptr;
 
     ZeroParams z;
     std::memset(&z, 0, sizeof z);
@@ -256,7 +272,7 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         rp.amax_row = (do_row && !nv) ? amax_row : nullptr;
         rp.q_row = q_row;
         rp.sf_row = sf_row;
-        rp.amax_col = (do_col && !colmax) ? amax_col : nullptr;
+        rp.amax_col = (do_col && !colmax && !xf_amax) ? amax_col : nullptr;
         rp.colmax = reinterpret_cast<uint32_t*>(colmax);
         rp.obs = absmax ? ws_obs(ws) : nullptr;
         for (int g = 0; g <= G; ++g) rp.row_off[g] = (int32_t)off[g];
@@ -267,11 +283,21 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         // With nothing to encode it runs the running-buffer update alone (one CTA).
         ColParams<MAXG> cp;
         std::memset(&cp, 0, sizeof cp);
+        // 512-row tasks (whole 32-byte sectors of column scales) unless that leaves fewer
+        // than two tasks per warp of the grid; then 256-row tasks
+        const int64_t strips = (cols + kTaskCols - 1) / kTaskCols;
+        auto count_tasks = [&](int32_t tr) {
+            int64_t t = 0;
+            for (int g = 0; g < G; ++g) t += (off[g + 1] - off[g] + tr - 1) / tr;
+            return t;
+        };
+        cp.task_rows = count_tasks(kTaskRows) * strips >= 2 * (int64_t)dev->sm_count * kColWarps ? kTaskRows
+                                                                                                 : kHalfRows;
         int32_t tasks = 0;
         for (int g = 0; g < G; ++g) {
             cp.row_off[g] = (int32_t)off[g];
             cp.task_off[g] = tasks;
-            tasks += (int32_t)((off[g + 1] - off[g] + kTaskRows - 1) / kTaskRows);
+            tasks += (int32_t)((off[g + 1] - off[g] + cp.task_rows - 1) / cp.task_rows);
         }
         cp.row_off[G] = (int32_t)off[G];
         cp.task_off[G] = tasks;
@@ -300,6 +326,25 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         cp.sf_col = sf_col;
         cp.absmax = absmax;
         cp.obs = ws_obs(ws);
+        if (opts) {
+            cp.rht = co->rht;
+            cp.rht_signs = co->rht_signs & 0xFFFFu;
+            cp.sr = co->sr;
+            cp.sr_key0 = (uint32_t)co->seed;
+            cp.sr_key1 = (uint32_t)(co->seed >> 32);
+            cp.sr_off0 = (uint32_t)co->offset;
+            cp.sr_off1 = (uint32_t)(co->offset >> 32);
+            if (xf_amax) {
+                ColParams<MAXG> ap = cp;
+                ap.absmax = nullptr;
+                ap.nbuf = 0;
+                if (launch(colpass<MAXG, false, kColXformAmax>, ap.num_ctas, 0, stream, ap, true, kColThreads) !=
+                    cudaSuccess)
+                    return NVFP4PT_ERR_CUDA;
+            }
+            e = launch(colpass<MAXG, false, kColOpts>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
+            return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+        }
         e = nv ? launch(colpass<MAXG, true>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads)
                : launch(colpass<MAXG, false>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
         return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
@@ -485,6 +530,29 @@ nvfp4pt_status quantize_grouped_ws(const void* x, int64_t rows, int64_t cols, co
 }  // namespace nvfp4pt
 
 extern "C" {
+
+nvfp4pt_status nvfp4pt_quantize_grouped_opts(const void* x, int64_t rows, int64_t cols, const int64_t* offsets,
+                                             int num_groups, int flags, uint8_t* q_row, uint8_t* sf_row,
+                                             float* amax_row, uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                                             float* absmax_bufs, float decay, const nvfp4pt_colwise_options* opts,
+                                             void* workspace, cudaStream_t stream)
+{
+    nvfp4pt_status st = nvfp4pt::check_grouped_args(x, rows, cols, offsets, num_groups, flags, q_row, sf_row,
+                                                    amax_row, q_col, sf_col, amax_col, absmax_bufs, workspace, true);
+    if (st != NVFP4PT_OK) return st;
+    ColOptions co = {};
+    if (opts) {
+        if (opts->flags & ~(NVFP4PT_COL_RHT | NVFP4PT_COL_SR)) return NVFP4PT_ERR_FLAGS;
+        co.rht = (opts->flags & NVFP4PT_COL_RHT) != 0;
+        co.sr = (opts->flags & NVFP4PT_COL_SR) != 0;
+        co.rht_signs = opts->rht_signs;
+        co.seed = opts->sr_seed;
+        co.offset = opts->sr_offset;
+        if ((co.rht || co.sr) && (flags & NVFP4PT_COLWISE) && cols > kRowPassMaxCols) return NVFP4PT_ERR_SHAPE;
+    }
+    return run_cast<kMaxGroups>(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row, q_col, sf_col,
+                                amax_col, absmax_bufs, decay, false, workspace, stream, nullptr, true, nullptr, &co);
+}
 
 nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w, int64_t rows, int64_t cols, uint8_t* q_row,
                                           uint8_t* sf_row, float* amax_row, void* workspace, cudaStream_t stream)

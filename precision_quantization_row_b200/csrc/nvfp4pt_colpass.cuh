@@ -24,13 +24,14 @@
 #pragma once
 
 #include "nvfp4pt_dequant.cuh"
+#include "nvfp4pt_xform.cuh"
 
 namespace nvfp4pt {
 
 constexpr int kColThreads = 512;   // one CTA per SM: 128 registers per thread
 constexpr int kColWarps = kColThreads / 32;
 constexpr int kStepRows = 64;      // rows of a step: four 16-row blocks
-constexpr int kTaskRows = 512;     // rows of a task: up to eight steps
+constexpr int kTaskRows = 512;     // rows of a task: up to eight steps (256 when tasks would be few)
 constexpr int kHalfRows = 256;     // rows whose codes are staged and written at once
 constexpr int kTaskCols = 32;      // columns of a task: 8 quads x 4
 constexpr int kColStageBytes = kTaskCols * (128 + 32);      // per warp: codes of a half, scales of a task
@@ -40,6 +41,7 @@ template <int MAXG>
 struct ColParams {
     int64_t cols;
     int64_t num_tasks;   // row tasks x strips
+    int32_t task_rows;   // rows of a task: kTaskRows, or kHalfRows when that leaves warps idle
     int32_t strips;      // ceil(cols / 32)
     int32_t num_ctas;
     int32_t num_groups;
@@ -62,9 +64,21 @@ struct ColParams {
     uint8_t* sf_col;
     float* absmax;           // [nbuf] running amax buffers, or null
     const float* obs;        // [G] amax observed by the row pass
+    // columnwise options (nvfp4pt_xform.cuh): the Hadamard transform with its sign mask,
+    // stochastic rounding with its Philox key and counter offset
+    int32_t rht;
+    uint32_t rht_signs;
+    int32_t sr;
+    uint32_t sr_key0, sr_key1, sr_off0, sr_off1;
     int32_t row_off[MAXG + 1];    // first row of each group
     int32_t task_off[MAXG + 1];   // first row task of each group
 };
+
+// What the column pass does with its tasks: the plain columnwise encode, the encode
+// with the columnwise options (the values of each block transformed and/or rounded
+// stochastically), or a sweep that only finds the column amax of the transformed values
+// (atomic max on the float bits into amax_col, which starts at zero).
+enum ColMode { kColPlain = 0, kColOpts = 1, kColXformAmax = 2 };
 
 // Codes of 8 consecutive rows of one column with one multiplier; the column is the
 // low (HI = false) or high half of the bf16 words v[r0 .. r0+7][w]. Row i -> bits 4i.
@@ -82,12 +96,35 @@ __device__ __forceinline__ uint32_t encode8_strided(const uint32_t (&v)[16][2], 
 
 // Where a task sits: its group, first row, row count and first column.
 struct ColTask {
+    int32_t g;        // token group
     int32_t row0;
     int32_t goff;
     int32_t grows;
     int32_t c0;
     int32_t nrows;    // 16..512, a multiple of 16
 };
+
+// Undo the staging order of a column's 32 scale bytes: position p of the row (p = 0..7
+// over the words of s0, s1) holds word p ^ x of the column.
+__device__ __forceinline__ void unswizzle_words(uint4& s0, uint4& s1, int x)
+{
+    uint32_t w[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int b = 1; b < 8; b <<= 1) {
+        if (x & b) {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                if ((p & b) == 0) {
+                    const uint32_t t = w[p];
+                    w[p] = w[p | b];
+                    w[p | b] = t;
+                }
+            }
+        }
+    }
+    s0 = make_uint4(w[0], w[1], w[2], w[3]);
+    s1 = make_uint4(w[4], w[5], w[6], w[7]);
+}
 
 // Staging slot of 8-byte chunk k (16 rows) of column c: 16-byte chunk (k >> 1) ^ g(c)
 // of the column's 128-byte row. g keeps both the lanes' 8-byte stores of a step and
@@ -111,8 +148,8 @@ __device__ __forceinline__ int group_of_task(const ColParams<MAXG>& p, int rt)
 }
 
 // NV = false: x is bf16. NV = true: the rows come dequantized from NVFP4 rowwise data
-// (nq, nsf, dscale), to the same bf16 values nvfp4pt_dequantize gives.
-template <int MAXG, bool NV = false>
+// (nq, nsf, dscale), to the same bf16 values nvfp4pt_dequantize gives. MODE: ColMode.
+template <int MAXG, bool NV = false, int MODE = kColPlain>
 __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant__ ColParams<MAXG> p)
 {
     // per warp: codes [column][16 chunks of 8 bytes] (swizzled), then scales [column][32]
@@ -149,11 +186,12 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
         if (MAXG > 1) {
             while (g > 0 && rt < p.task_off[g]) --g;
         }
+        ct.g = g;
         ct.goff = p.row_off[g];
         ct.grows = p.row_off[g + 1] - ct.goff;
-        ct.row0 = ct.goff + (rt - p.task_off[g]) * kTaskRows;
+        ct.row0 = ct.goff + (rt - p.task_off[g]) * p.task_rows;
         const int left = ct.goff + ct.grows - ct.row0;
-        ct.nrows = left >= kTaskRows ? kTaskRows : left;
+        ct.nrows = left >= p.task_rows ? p.task_rows : left;
         ct.c0 = strip * kTaskCols;
     };
     auto step_back = [&]() {
@@ -228,7 +266,7 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
     }
 
     griddep_wait();
-    if (blockIdx.x == 0 && p.absmax) {
+    if (MODE != kColXformAmax && blockIdx.x == 0 && p.absmax) {
         for (int i = tid; i < p.nbuf; i += kColThreads) {
             const float d = __fmul_rn(p.absmax[i], p.decay);
             const float o = p.obs[i];
@@ -243,11 +281,13 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
     // This lane's slots: column 4q+j, block kb = 4*(step & 3) + blk of the current half
     // goes to stage_off(4q+j, kb) = xq + 128j + 16*(hg ^ j), hg = (kb >> 1) ^ G(q), where
     // g(4q+j) = j ^ G(q) with G(q) = 4(q & 1) ^ (q & 6); its scale byte (block
-    // 4*step + blk of the task) to xsq + 32j + 4*step.
+    // 4*step + blk of the task) to column 4q+j's 32-byte row at word (step ^ q), byte
+    // blk: the scale stores of a step then fall on eight different banks.
     uint8_t* xq = xc + 512 * quad + 8 * (blk & 1);
     uint8_t* xsq = xs + 128 * quad + blk;
     const int gq = (4 * (quad & 1)) ^ (quad & 6);
     const uint64_t pol_out = l2_evict_first();
+    float xamax[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // kColXformAmax: this lane's column maxima of the task
     float sc[4];
     {
         const float a = load_amax(cur);
@@ -291,37 +331,92 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
             }
         }
 
-        // block amax of the four columns over this lane's 16 rows
-        uint32_t m[2];
+        if constexpr (MODE == kColPlain) {
+            // block amax of the four columns over this lane's 16 rows
+            uint32_t m[2];
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            uint32_t t[8];
+            for (int w = 0; w < 2; ++w) {
+                uint32_t t[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) t[i] = absmax2(v[i][w], v[i + 8][w]);
+                for (int i = 0; i < 8; ++i) t[i] = absmax2(v[i][w], v[i + 8][w]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) t[i] = absmax2(t[i], t[i + 4]);
-            t[0] = absmax2(t[0], t[2]);
-            t[1] = absmax2(t[1], t[3]);
-            m[w] = absmax2(t[0], t[1]) & 0x7FFF7FFFu;
-        }
-        uint32_t sf01, sf23;
-        float e[4];
-        block_pair_scales_x2(bf16_lo(m[0]), bf16_hi(m[0]), sc[0], sc[1], sf01, e[0], e[1], rcp_tab);
-        block_pair_scales_x2(bf16_lo(m[1]), bf16_hi(m[1]), sc[2], sc[3], sf23, e[2], e[3], rcp_tab);
+                for (int i = 0; i < 4; ++i) t[i] = absmax2(t[i], t[i + 4]);
+                t[0] = absmax2(t[0], t[2]);
+                t[1] = absmax2(t[1], t[3]);
+                m[w] = absmax2(t[0], t[1]) & 0x7FFF7FFFu;
+            }
+            uint32_t sf01, sf23;
+            float e[4];
+            block_pair_scales_x2(bf16_lo(m[0]), bf16_hi(m[0]), sc[0], sc[1], sf01, e[0], e[1], rcp_tab);
+            block_pair_scales_x2(bf16_lo(m[1]), bf16_hi(m[1]), sc[2], sc[3], sf23, e[2], e[3], rcp_tab);
 
-        // codes and scales of this lane's block of each column -> staging
-        const int hg = (2 * (step & 3) + (blk >> 1)) ^ gq;
-        uint8_t* xsb = xsq + 4 * step;
+            // codes and scales of this lane's block of each column -> staging
+            const int hg = (2 * (step & 3) + (blk >> 1)) ^ gq;
+            uint8_t* xsb = xsq + 4 * (step ^ quad);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int w = j >> 1;
-            const uint32_t lo = (j & 1) ? encode8_strided<true>(v, 0, w, e[j]) : encode8_strided<false>(v, 0, w, e[j]);
-            const uint32_t hi = (j & 1) ? encode8_strided<true>(v, 8, w, e[j]) : encode8_strided<false>(v, 8, w, e[j]);
-            *reinterpret_cast<uint2*>(xq + 128 * j + 16 * (hg ^ j)) = make_uint2(lo, hi);
-            xsb[32 * j] = (uint8_t)(((j < 2) ? sf01 : sf23) >> (8 * (j & 1)));
+            for (int j = 0; j < 4; ++j) {
+                const int w = j >> 1;
+                const uint32_t lo = (j & 1) ? encode8_strided<true>(v, 0, w, e[j]) : encode8_strided<false>(v, 0, w, e[j]);
+                const uint32_t hi = (j & 1) ? encode8_strided<true>(v, 8, w, e[j]) : encode8_strided<false>(v, 8, w, e[j]);
+                *reinterpret_cast<uint2*>(xq + 128 * j + 16 * (hg ^ j)) = make_uint2(lo, hi);
+                xsb[32 * j] = (uint8_t)(((j < 2) ? sf01 : sf23) >> (8 * (j & 1)));
+            }
+        } else {
+            // one column at a time: its 16 values as binary32, the transform, the block
+            // steps with IEEE divisions, codes by nearest or stochastic rounding
+            const int hg = (2 * (step & 3) + (blk >> 1)) ^ gq;
+            uint8_t* xsb = xsq + 4 * (step ^ quad);
+            const int64_t m0 = (int64_t)cur.row0 + kStepRows * step + 16 * blk;   // first row of the block
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float f[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) f[i] = (j & 1) ? bf16_hi(v[i][j >> 1]) : bf16_lo(v[i][j >> 1]);
+                if (p.rht) rht16(f, p.rht_signs);
+                float ba = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ba = fmaxf(ba, fabsf(f[i]));
+                if constexpr (MODE == kColXformAmax) {
+                    xamax[j] = fmaxf(xamax[j], ba);
+                } else {
+                    uint32_t sf;
+                    float e;
+                    block_scale_ieee(ba, sc[j], sf, e);
+                    float y[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(f[i], e);
+                    uint32_t lo = 0u, hi = 0u;
+                    if (p.sr) {
+                        const uint32_t col = (uint32_t)(cur.c0 + 4 * quad + j);
+#pragma unroll
+                        for (int t4 = 0; t4 < 4; ++t4) {
+                            const uint4 r = philox10((uint32_t)((m0 >> 2) + t4), col, p.sr_off0, p.sr_off1,
+                                                     p.sr_key0, p.sr_key1);
+                            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int i = 4 * t4 + u;
+                                const uint32_t code = e2m1_sr(y[i], rw[u]);
+                                if (i < 8) lo |= code << (4 * i); else hi |= code << (4 * (i - 8));
+                            }
+                        }
+                    } else {
+                        float ylo[8], yhi[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            ylo[i] = y[i];
+                            yhi[i] = y[i + 8];
+                        }
+                        lo = e2m1x8_packed(ylo);
+                        hi = e2m1x8_packed(yhi);
+                    }
+                    *reinterpret_cast<uint2*>(xq + 128 * j + 16 * (hg ^ j)) = make_uint2(lo, hi);
+                    xsb[32 * j] = (uint8_t)sf;
+                }
+            }
         }
 
-        if ((step & 3) == 0) {
+        if (MODE != kColXformAmax && (step & 3) == 0) {
             // a half done: write its codes out of staging (the half's rows start at
             // 64 * step of the task)
             __syncwarp();
@@ -357,26 +452,45 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
             __syncwarp();   // staging is written again by the next step
         }
         if (step == 0) {
-            // task done: lane j writes column j's block scales, one whole 32-byte sector
-            // per column when the task has 512 rows
-            const int nblk = cur.nrows / 16;
-            const int lrow = cur.row0 - cur.goff;
-            const int c = cur.c0 + lane;
-            if (c < cols) {
-                uint8_t* sf = p.sf_col + cols * cur.goff / 16 + (int64_t)c * (cur.grows / 16) + lrow / 16;
-                const uint4 s0 = *reinterpret_cast<const uint4*>(xs + 32 * lane);
-                const uint4 s1 = *reinterpret_cast<const uint4*>(xs + 32 * lane + 16);
-                const uintptr_t al = reinterpret_cast<uintptr_t>(sf);
-                if (nblk == 32 && (al & 31u) == 0) {
-                    stg32_ef(sf, s0, s1, pol_out);
-                } else if (nblk == 32 && (al & 15u) == 0) {
-                    stg16_ef(sf, s0, pol_out);
-                    stg16_ef(sf + 16, s1, pol_out);
-                } else {
-                    const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            if constexpr (MODE == kColXformAmax) {
+                // task done: the four lanes of each column quad combine their maxima and
+                // one of them raises the task's group's amax_col entries (the walk's g
+                // already names the next task's group)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (4 * i < nblk) stg_bytes(sf + 4 * i, sw[i], min(4, nblk - 4 * i));
+                for (int j = 0; j < 4; ++j) {
+                    float a = fmaxf(xamax[j], __shfl_xor_sync(0xFFFFFFFFu, xamax[j], 8));
+                    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 16));
+                    const int c = cur.c0 + 4 * quad + j;
+                    if (blk == 0 && c < cols && a > 0.0f)
+                        red_max_f32(p.amax_col + (int64_t)cur.g * cols + c, __float_as_uint(a));
+                    xamax[j] = 0.0f;
+                }
+            } else {
+                // task done: lane j writes column j's block scales, one whole 32-byte sector
+                // per column when the task has 512 rows
+                const int nblk = cur.nrows / 16;
+                const int lrow = cur.row0 - cur.goff;
+                const int c = cur.c0 + lane;
+                if (c < cols) {
+                    uint8_t* sf = p.sf_col + cols * cur.goff / 16 + (int64_t)c * (cur.grows / 16) + lrow / 16;
+                    // the row's word at position w ^ (lane >> 2) is the column's word w
+                    uint4 s0 = *reinterpret_cast<const uint4*>(xs + 32 * lane);
+                    uint4 s1 = *reinterpret_cast<const uint4*>(xs + 32 * lane + 16);
+                    unswizzle_words(s0, s1, lane >> 2);
+                    const uintptr_t al = reinterpret_cast<uintptr_t>(sf);
+                    if (nblk == 32 && (al & 31u) == 0) {
+                        stg32_ef(sf, s0, s1, pol_out);
+                    } else if (nblk == 32 && (al & 15u) == 0) {
+                        stg16_ef(sf, s0, pol_out);
+                        stg16_ef(sf + 16, s1, pol_out);
+                    } else if (nblk == 16 && (al & 15u) == 0) {
+                        stg16_ef(sf, s0, pol_out);
+                    } else {
+                        const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (4 * i < nblk) stg_bytes(sf + 4 * i, sw[i], min(4, nblk - 4 * i));
+                    }
                 }
             }
             __syncwarp();

@@ -2,6 +2,7 @@
 // TMA descriptors of the operands and the launch of the tcgen05 kernel.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -18,6 +19,13 @@ constexpr int kMaxDevices = 64;
 
 std::mutex g_mu;
 bool g_ready[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+
+int dev_index()
+{
+    int dev = 0;
+    return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices ? dev : 0;
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -38,7 +46,8 @@ nvfp4pt_status gemm_setup()
     }
     if (!g_ready[dev]) {
         if (cudaFuncSetAttribute(gemm_per_token_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || g_sms[dev] < 1)
             return NVFP4PT_ERR_CUDA;
         g_ready[dev] = true;
     }
@@ -96,9 +105,12 @@ nvfp4pt_status nvfp4pt_gemm_per_token(const uint8_t* qa, const uint8_t* sfa, con
     p.d = d;
     p.err = static_cast<uint32_t*>(workspace);
     if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess) return NVFP4PT_ERR_CUDA;
-    const int64_t tiles = ((m + kGemmBM - 1) / kGemmBM) * ((n + kGemmBN - 1) / kGemmBN);
+    p.m_tiles = (int32_t)((m + kGemmBM - 1) / kGemmBM);
     p.n_tiles = (int32_t)((n + kGemmBN - 1) / kGemmBN);
-    gemm_per_token_kernel<<<(unsigned)tiles, kGemmThreads, kGemmSmem, stream>>>(p);
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    // one persistent CTA per SM (or per tile, when there are fewer tiles)
+    const int grid = (int)std::min<int64_t>(tiles, g_sms[dev_index()]);
+    gemm_per_token_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 

@@ -9,17 +9,19 @@
 // (TransformerEngine PR #3045 "Add NVFP4 per-token quantization recipe": a GEMM that
 // rescales with the per-row and per-column outer-amax vectors inside its epilogue).
 //
-// One CTA computes a 128 x 256 tile of D:
+// A persistent CTA per SM takes 128 x 256 tiles of D in turn:
 //   warp 0       TMA producer: per 256-element K step, the A and B code tiles (128-byte
-//                rows, 128-byte swizzle) and the A and B block-scale rows (16 bytes each).
-//   warp 1       allocates tensor memory; its lanes move the block scales into the
-//                layout the scale copy reads, and lane 0 issues the scale copies into
+//                rows, 128-byte swizzle) and the A and B block-scale rows (16 bytes
+//                each), four stages deep, running ahead into the next tile.
+//   warp 1       allocates tensor memory; its lanes rearrange the block scales in place
+//                into the layout of the scale copy, and lane 0 issues the copies into
 //                tensor memory (tcgen05.cp) and the four block-scaled MMAs of the step
 //                (tcgen05.mma kind::mxf4nvf4, 16-element E4M3 scale vectors).
-//   warps 4..7   epilogue: the fp32 accumulator from tensor memory (tcgen05.ld), times
-//                S_dec(a_m), times S_dec(b_n), to D (fp32, row-major).
-// Every wait on an mbarrier is bounded; a wait that gives up sets the error word and the
-// CTA skips the rest of its work (after its copies in flight have landed).
+//   warps 2..9   epilogue: each drains 32 rows x 128 columns of the fp32 accumulator
+//                into registers (tcgen05.ld) and frees it, so the next tile's MMAs run
+//                while it multiplies by S_dec(a_m) and S_dec(b_n) and stores D.
+// Every wait on an mbarrier is bounded; a wait that gives up sets the error word and
+// the warp skips the rest of its work (after its copies in flight have landed).
 #pragma once
 
 #include "nvfp4pt_device.cuh"
@@ -29,19 +31,18 @@ namespace nvfp4pt {
 constexpr int kGemmBM = 128;           // rows of A per tile (the MMA's M)
 constexpr int kGemmBN = 256;           // rows of B per tile (the MMA's N)
 constexpr int kGemmBK = 256;           // K elements per pipeline stage: one 128-byte row of codes
-constexpr int kGemmStages = 3;
-constexpr int kGemmThreads = 256;      // 8 warps; warps 2 and 3 only join the barriers
+constexpr int kGemmStages = 4;
+constexpr int kGemmEpiWarps = 8;       // two per 32-lane group of tensor memory, 128 columns each
+constexpr int kGemmThreads = 32 * (2 + kGemmEpiWarps);
 constexpr int kGemmTmemCols = 512;     // accumulator 256 columns + scale factors 48
 
 // shared memory of one stage (offsets from the 1024-aligned stage base)
 constexpr int kGsA = 0;                               // A codes  128 x 128 B
 constexpr int kGsB = kGsA + kGemmBM * 128;            // B codes  256 x 128 B
-constexpr int kGsSfaRaw = kGsB + kGemmBN * 128;       // A scales 128 x 16 B, as loaded
-constexpr int kGsSfbRaw = kGsSfaRaw + kGemmBM * 16;   // B scales 256 x 16 B, as loaded
-constexpr int kGsSfa = kGsSfbRaw + kGemmBN * 16;      // A scales in copy layout, 4 x 512 B
-constexpr int kGsSfb = kGsSfa + kGemmBM * 16;         // B scales in copy layout, 8 x 512 B
+constexpr int kGsSfa = kGsB + kGemmBN * 128;          // A scales 128 x 16 B, then in copy layout
+constexpr int kGsSfb = kGsSfa + kGemmBM * 16;         // B scales 256 x 16 B, then in copy layout
 constexpr int kGemmStageBytes = kGsSfb + kGemmBN * 16;
-constexpr int kGemmTxBytes = kGsSfa;                  // bytes the TMA brings per stage
+constexpr int kGemmTxBytes = kGemmStageBytes;         // bytes the TMA brings per stage
 constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024;   // + room to align the stages to 1024
 
 // tensor memory columns (lane field 0)
@@ -59,7 +60,8 @@ struct GemmParams {
     const float* amax_b;
     float* d;            // [M, N] fp32
     uint32_t* err;
-    int32_t n_tiles;     // tiles along N; CTA t takes tile (t / n_tiles, t % n_tiles)
+    int32_t m_tiles;     // tiles along M
+    int32_t n_tiles;     // tiles along N; tile t is (t / n_tiles, t % n_tiles), CTA c takes c, c + grid, ...
 };
 
 // Block-scaled MMA instruction descriptor: E2M1 A and B (K-major), E4M3 scales, fp32
@@ -133,8 +135,9 @@ __device__ __forceinline__ void tc_commit(uint32_t bar)
                  : "memory");
 }
 
-// 32 consecutive fp32 columns of this warp's 32 lanes: lane i gets row (base lane + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+// 32 consecutive fp32 columns of this warp's 32 lanes: lane i gets row (base lane + i);
+// the registers are valid after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
                  "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -145,35 +148,45 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
                    "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
                    "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
                  : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Rows [row0, row0 + 32 * nblk) of a [rows][16 B] scale tile into the copy layout: for each
-// of the four MMA K steps kb, blocks of 512 bytes, one per 128 rows, whose 16-byte line i
-// holds the kb-th scale word (4 scales) of rows i, i + 32, i + 64, i + 96. Lane i of a warp.
-__device__ __forceinline__ void sf_to_copy_layout(uint32_t raw, uint32_t dst, int lane, int nblk)
+// A [128 * nblk][16 B] scale tile, rearranged in place into the copy layout: 128-row
+// block b becomes four 512-byte pieces at b * 2048 + kb * 512 (kb: the MMA K step),
+// whose 16-byte line i holds the kb-th scale word (4 scales) of the block's rows i,
+// i + 32, i + 64, i + 96. A block's pieces take exactly its own 2048 bytes, so the
+// warp reads a block whole before it writes it. Lane i of a warp.
+__device__ __forceinline__ void sf_to_copy_layout(uint32_t base, int lane, int nblk)
 {
     for (int b = 0; b < nblk; ++b) {
+        const uint32_t blk = base + 2048u * (uint32_t)b;
         uint4 r[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) r[c] = lds128(raw + 16u * (uint32_t)(128 * b + 32 * c + lane));
+        for (int c = 0; c < 4; ++c) r[c] = lds128(blk + 16u * (uint32_t)(32 * c + lane));
+        __syncwarp();
         const uint32_t w0[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
         const uint32_t w1[4] = {r[1].x, r[1].y, r[1].z, r[1].w};
         const uint32_t w2[4] = {r[2].x, r[2].y, r[2].z, r[2].w};
         const uint32_t w3[4] = {r[3].x, r[3].y, r[3].z, r[3].w};
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t a = dst + 512u * (uint32_t)(kb * nblk + b) + 16u * (uint32_t)lane;
+            const uint32_t a = blk + 512u * (uint32_t)kb + 16u * (uint32_t)lane;
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0[kb]), "r"(w1[kb]),
                          "r"(w2[kb]), "r"(w3[kb])
                          : "memory");
         }
     }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void gemm_fail(uint32_t* err, uint32_t code)
@@ -184,36 +197,31 @@ __device__ __forceinline__ void gemm_fail(uint32_t* err, uint32_t code)
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const __grid_constant__ GemmParams p)
 {
     extern __shared__ __align__(1024) uint8_t gemm_smem_raw[];
-    __shared__ __align__(8) uint64_t bar_mem[2 * kGemmStages + 1];   // full[S], empty[S], acc_full
+    // full[S], empty[S], acc_full, acc_empty
+    __shared__ __align__(8) uint64_t bar_mem[2 * kGemmStages + 2];
     __shared__ uint32_t tmem_slot_mem;
-    __shared__ float sdec_b[kGemmBN];                                // S_dec(b_n) of the tile's columns
     const uint32_t smem0 = (smem_u32(gemm_smem_raw) + 1023u) & ~1023u;
-    const uint32_t full0 = smem_u32(bar_mem), empty0 = full0 + 8 * kGemmStages, acc_bar = full0 + 16 * kGemmStages;
-    const uint32_t tmem_slot = smem_u32(&tmem_slot_mem);
+    const uint32_t full0 = smem_u32(bar_mem), empty0 = full0 + 8 * kGemmStages;
+    const uint32_t acc_full = full0 + 16 * kGemmStages, acc_empty = acc_full + 8;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = (int64_t)(blockIdx.x / p.n_tiles) * kGemmBM;
-    const int64_t n0 = (int64_t)(blockIdx.x % p.n_tiles) * kGemmBN;
     const int ksteps = (int)(p.k / kGemmBK);
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
-        mbar_init(acc_bar, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kGemmEpiWarps);
         fence_mbar_init();
         prefetch_tensormap(&p.tmA);
         prefetch_tensormap(&p.tmB);
         prefetch_tensormap(&p.tmSfa);
         prefetch_tensormap(&p.tmSfb);
     }
-    if (warp == 1) tmem_alloc(tmem_slot, kGemmTmemCols);
-    // the epilogue's column decode scales S_dec(b_n) = RN(amax_b[n] / 2688)
-    for (int j = (int)threadIdx.x; j < kGemmBN; j += kGemmThreads) {
-        const int64_t n = n0 + j;
-        sdec_b[j] = n < p.n ? __fdiv_rn(__ldg(p.amax_b + n), 2688.0f) : 0.0f;
-    }
+    if (warp == 1) tmem_alloc(smem_u32(&tmem_slot_mem), kGemmTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -222,100 +230,129 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         if (lane == 0) {
-            int issued = 0;
+            int64_t it = 0;   // K steps issued over all tiles
             bool ok = true;
-            for (int t = 0; t < ksteps && ok; ++t) {
-                const int s = t % kGemmStages;
-                const uint32_t ph = (uint32_t)((t / kGemmStages) & 1);
-                if (t >= kGemmStages && !mbar_wait_bounded(empty0 + 8 * s, ph ^ 1u)) {
-                    gemm_fail(p.err, kErrTmaTimeout);
-                    ok = false;
-                    break;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int32_t m0 = (int32_t)(t / p.n_tiles) * kGemmBM, n0 = (int32_t)(t % p.n_tiles) * kGemmBN;
+                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int s = (int)(it % kGemmStages);
+                    const uint32_t ph = (uint32_t)((it / kGemmStages) & 1);
+                    if (it >= kGemmStages && !mbar_wait_bounded(empty0 + 8 * s, ph ^ 1u)) {
+                        gemm_fail(p.err, kErrTmaTimeout);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = smem0 + s * kGemmStageBytes;
+                    const uint32_t fb = full0 + 8 * s;
+                    mbar_arrive_expect_tx(fb, kGemmTxBytes);
+                    tma_load_2d(st + kGsA, &p.tmA, ks * 128, m0, fb);
+                    tma_load_2d(st + kGsB, &p.tmB, ks * 128, n0, fb);
+                    tma_load_2d(st + kGsSfa, &p.tmSfa, ks * 16, m0, fb);
+                    tma_load_2d(st + kGsSfb, &p.tmSfb, ks * 16, n0, fb);
                 }
-                const uint32_t st = smem0 + s * kGemmStageBytes;
-                const uint32_t fb = full0 + 8 * s;
-                mbar_arrive_expect_tx(fb, kGemmTxBytes);
-                tma_load_2d(st + kGsA, &p.tmA, t * 128, (int32_t)m0, fb);
-                tma_load_2d(st + kGsB, &p.tmB, t * 128, (int32_t)n0, fb);
-                tma_load_2d(st + kGsSfaRaw, &p.tmSfa, t * 16, (int32_t)m0, fb);
-                tma_load_2d(st + kGsSfbRaw, &p.tmSfb, t * 16, (int32_t)n0, fb);
-                issued = t + 1;
             }
             // copies must not land in freed shared memory: wait for the last ones issued
-            for (int t = issued - kGemmStages > 0 ? issued - kGemmStages : 0; t < issued; ++t) {
-                const int s = t % kGemmStages;
-                if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)((t / kGemmStages) & 1)))
+            for (int64_t j = it - kGemmStages > 0 ? it - kGemmStages : 0; j < it; ++j) {
+                const int s = (int)(j % kGemmStages);
+                if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)((j / kGemmStages) & 1)))
                     gemm_fail(p.err, kErrDrainTimeout);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ scale layout + MMA issue
         const uint32_t idesc = gemm_idesc();
-        for (int t = 0; t < ksteps; ++t) {
-            const int s = t % kGemmStages;
-            const uint32_t ph = (uint32_t)((t / kGemmStages) & 1);
-            // the whole warp leaves together if any lane's wait gave up
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full0 + 8 * s, ph))) {
+        int64_t it = 0;
+        int j = 0;    // tiles of this CTA so far
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+            // the epilogue has drained the previous tile's accumulator
+            if (j > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_empty, (uint32_t)((j - 1) & 1)))) {
                 if (lane == 0) gemm_fail(p.err, kErrTmaTimeout);
                 break;
             }
-            const uint32_t st = smem0 + s * kGemmStageBytes;
-            sf_to_copy_layout(st + kGsSfaRaw, st + kGsSfa, lane, kGemmBM / 128);
-            sf_to_copy_layout(st + kGsSfbRaw, st + kGsSfb, lane, kGemmBN / 128);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    tmem_cp_sf(tbase + kTmSfa + 4 * kb, smem_desc_sf(st + kGsSfa + 512 * kb));
-#pragma unroll
-                    for (int h = 0; h < kGemmBN / 128; ++h)
-                        tmem_cp_sf(tbase + kTmSfb + 8 * kb + 4 * h,
-                                   smem_desc_sf(st + kGsSfb + 512 * (kb * (kGemmBN / 128) + h)));
+            tc_fence_after();
+            for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                const int s = (int)(it % kGemmStages);
+                const uint32_t ph = (uint32_t)((it / kGemmStages) & 1);
+                // the whole warp leaves together if any lane's wait gave up
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full0 + 8 * s, ph))) {
+                    if (lane == 0) gemm_fail(p.err, kErrTmaTimeout);
+                    ok = false;
+                    break;
                 }
+                const uint32_t st = smem0 + s * kGemmStageBytes;
+                sf_to_copy_layout(st + kGsSfa, lane, kGemmBM / 128);
+                sf_to_copy_layout(st + kGsSfb, lane, kGemmBN / 128);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
 #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    // K step kb of the stage: 64 codes = 32 bytes into each 128-byte row
-                    const uint64_t ad = smem_desc_sw128(st + kGsA + 32 * kb);
-                    const uint64_t bd = smem_desc_sw128(st + kGsB + 32 * kb);
-                    mma_fp4_block16(tbase + kTmAcc, ad, bd, idesc, tbase + kTmSfa + 4 * kb, tbase + kTmSfb + 8 * kb,
-                                    (t > 0 || kb > 0) ? 1u : 0u);
-                }
-                tc_commit(empty0 + 8 * s);   // the stage's shared memory is free once these finish
-            }
-            __syncwarp();
-        }
-        if (lane == 0) tc_commit(acc_bar);   // all MMAs issued above (or none) have completed
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------- epilogue
-        const int q = warp & 3;                 // this warp's 32-lane group of tensor memory
-        const int64_t row = m0 + 32 * q + lane;
-        const bool ok = mbar_wait_bounded(acc_bar, 0);
-        if (!ok) gemm_fail(p.err, kErrTmaTimeout);
-        tc_fence_after();
-        const uint32_t err_now = *reinterpret_cast<volatile uint32_t*>(p.err);
-        // tcgen05.ld is warp-collective: the warp reads the accumulator only if every lane may
-        if (__all_sync(0xFFFFFFFFu, ok && err_now == 0)) {
-            const float sa = row < p.m ? __fdiv_rn(__ldg(p.amax_a + row), 2688.0f) : 0.0f;
-            for (int c0 = 0; c0 < kGemmBN; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(tbase + ((uint32_t)(32 * q) << 16) + kTmAcc + (uint32_t)c0, v);
-                if (row < p.m && n0 + c0 < p.n) {
-                    float* dst = p.d + row * p.n + n0 + c0;
-                    const int nc = (int)(p.n - (n0 + c0) < 32 ? p.n - (n0 + c0) : 32);   // a multiple of 16
+                    for (int kb = 0; kb < 4; ++kb) {
+                        tmem_cp_sf(tbase + kTmSfa + 4 * kb, smem_desc_sf(st + kGsSfa + 512 * kb));
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        if (4 * j4 < nc) {
-                            float o[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const int j = 4 * j4 + u;
-                                o[u] = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), sa), sdec_b[c0 + j]);
-                            }
-                            *reinterpret_cast<float4*>(dst + 4 * j4) = make_float4(o[0], o[1], o[2], o[3]);
-                        }
+                        for (int h = 0; h < kGemmBN / 128; ++h)
+                            tmem_cp_sf(tbase + kTmSfb + 8 * kb + 4 * h,
+                                       smem_desc_sf(st + kGsSfb + 2048 * h + 512 * kb));
                     }
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        // K step kb of the stage: 64 codes = 32 bytes into each 128-byte row
+                        const uint64_t ad = smem_desc_sw128(st + kGsA + 32 * kb);
+                        const uint64_t bd = smem_desc_sw128(st + kGsB + 32 * kb);
+                        mma_fp4_block16(tbase + kTmAcc, ad, bd, idesc, tbase + kTmSfa + 4 * kb,
+                                        tbase + kTmSfb + 8 * kb, (ks > 0 || kb > 0) ? 1u : 0u);
+                    }
+                    tc_commit(empty0 + 8 * s);   // the stage's shared memory is free once these finish
+                }
+                __syncwarp();
+            }
+            if (lane == 0) tc_commit(acc_full);   // the tile's accumulator is complete
+        }
+    } else {
+        // ------------------------------------------------------------- epilogue
+        const int q = warp & 3;                  // this warp's 32-lane group of tensor memory
+        const int half = (warp - 2) >> 2;        // and its 128 columns of the tile
+        int j = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const int64_t m0 = (t / p.n_tiles) * kGemmBM, n0 = (t % p.n_tiles) * kGemmBN + 128 * half;
+            const int64_t row = m0 + 32 * q + lane;
+            // the column decode scales S_dec(b_n) of this warp's 128 columns, 4 per lane
+            float sdec[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t n = n0 + 4 * lane + u;
+                sdec[u] = n < p.n ? __fdiv_rn(__ldg(p.amax_b + n), 2688.0f) : 0.0f;
+            }
+            const float sa = row < p.m ? __fdiv_rn(__ldg(p.amax_a + row), 2688.0f) : 0.0f;
+            const bool ok = mbar_wait_bounded(acc_full, (uint32_t)(j & 1));
+            if (!ok) gemm_fail(p.err, kErrTmaTimeout);
+            tc_fence_after();
+            // tcgen05.ld is warp-collective: the warp reads the accumulator only if every lane may
+            if (!__all_sync(0xFFFFFFFFu, ok && *reinterpret_cast<volatile uint32_t*>(p.err) == 0)) break;
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tmem_ld32_nowait(tbase + ((uint32_t)(32 * q) << 16) + kTmAcc + (uint32_t)(128 * half + 32 * c), v[c]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);   // the MMA warp may overwrite the accumulator
+            // every lane takes part in the shuffles; lanes past the last row store nothing
+            float* dst = p.d + row * p.n + n0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const int col = 32 * c + 4 * j4;       // column of the warp's 128
+                    float o[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float sb = __shfl_sync(0xFFFFFFFFu, sdec[u], col >> 2);
+                        o[u] = __fmul_rn(__fmul_rn(__uint_as_float(v[c][4 * j4 + u]), sa), sb);
+                    }
+                    if (row < p.m && n0 + col < p.n)
+                        *reinterpret_cast<float4*>(dst + col) = make_float4(o[0], o[1], o[2], o[3]);
                 }
             }
         }

@@ -68,6 +68,8 @@ def _worker(task):
         return kind, a, b, oracle.quantize(np.ascontiguousarray(x[a:b]), flags=COLWISE)
     if kind == "w2d":
         return kind, a, b, oracle.quantize_weight_2d(np.ascontiguousarray(x[a:b]))
+    if kind == "colopts":
+        return kind, a, b, oracle.quantize_colwise_opts(np.ascontiguousarray(x[:, a:b]), col_base=a, **extra)
     raise ValueError(kind)
 
 
@@ -128,6 +130,37 @@ def oracle_quantize_parallel(x: torch.Tensor, flags=ROWWISE | COLWISE, offsets=N
     if not flags & ROWWISE:
         out.pop("amax_row")
     return out
+
+
+def oracle_colwise_opts_parallel(x: torch.Tensor, offsets=None, parts=None, **opts) -> dict:
+    """The oracle's columnwise cast with the options (rht, rht_signs, sr, seed, offset) over
+    column ranges in a spawn pool: a column's outputs depend on that column alone (the
+    random words take its index in the full matrix). Outputs shaped as
+    oracle.quantize_colwise_opts's."""
+    xb = bits_of(x)
+    M, K = xb.shape
+    parts = parts or max(1, min(32, os.cpu_count() or 1)) * 2
+    G = 1 if offsets is None else len(offsets) - 1
+    off = [0, M] if offsets is None else [int(o) for o in offsets]
+    q = np.zeros(K * M // 2, np.uint8)
+    sf = np.zeros(K * M // 16, np.uint8)
+    am = np.zeros((G, K), np.float32)
+    with _scratch_dir() as d:
+        path = os.path.join(d, "x.npy")
+        np.save(path, xb)
+        tasks = [("colopts", path, a, b, dict(opts, offsets=off)) for a, b in _split(K, parts)]
+        with _pool(len(tasks)) as ex:
+            for kind, a, b, r in ex.map(_worker, tasks):
+                am[:, a:b] = r["amax_col"]
+                for g in range(G):
+                    r0, m = off[g], off[g + 1] - off[g]
+                    qg = r["q_col"][(b - a) * r0 // 2:(b - a) * (r0 + m) // 2].reshape(b - a, m // 2)
+                    sg = r["sf_col"][(b - a) * r0 // 16:(b - a) * (r0 + m) // 16].reshape(b - a, m // 16)
+                    q[K * r0 // 2 + a * (m // 2):K * r0 // 2 + b * (m // 2)] = qg.ravel()
+                    sf[K * r0 // 16 + a * (m // 16):K * r0 // 16 + b * (m // 16)] = sg.ravel()
+    if offsets is None:
+        return {"q_col": q.reshape(K, M // 2), "sf_col": sf.reshape(K, M // 16), "amax_col": am.reshape(K)}
+    return {"q_col": q, "sf_col": sf, "amax_col": am}
 
 
 def oracle_weight_2d_parallel(w: torch.Tensor, parts=None) -> dict:

@@ -190,6 +190,28 @@ def test_gemm_rejections(L):
     assert g() in (5, 6)
 
 
+def test_options_rejections(L):
+    import precision_quantization_row_b200 as nvp
+    h = _Host()
+    P = h.p
+
+    def o(flags=0, cols=32, rows=64, opt_flags=nvp.COL_RHT):
+        arr = (ctypes.c_int64 * 2)(0, rows)
+        opts = nvp.ColwiseOptions(opt_flags, 0xBEEF, 1, 2)
+        return L.nvfp4pt_quantize_grouped_opts(P(), rows, cols, arr, 1, flags or 3, *[P()] * 6, None, F0,
+                                               ctypes.byref(opts), P(), None)
+
+    assert o(opt_flags=4) == 7
+    assert o(opt_flags=8) == 7
+    assert o(cols=16400) == 2                       # options need rows of at most 16384 elements
+    assert o(cols=16400, flags=1) in (5, 6)         # ... only for the columnwise direction
+    assert o(cols=20) == 2
+    assert o() in (5, 6)
+    assert o(opt_flags=3) in (5, 6)
+    assert L.nvfp4pt_quantize_grouped_opts(P(), 64, 32, (ctypes.c_int64 * 2)(0, 64), 1, 3, *[P()] * 6, None, F0,
+                                           None, P(), None) in (5, 6)   # NULL options: the plain cast
+
+
 def test_probe_rejections():
     import probe
     PL = probe.lib()
