@@ -46,7 +46,7 @@ def workload_name(m: int, k: int) -> str:
 PROFILE_JSON = os.path.join(ROOT, "profiles", "nvfp4pt_cast_llm_16384x8192.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "precision_quantization_row_b200", "csrc", f)
                   for f in ("nvfp4pt_api.cu", "nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh", "nvfp4pt_rowpass.cuh",
-                            "nvfp4pt_colpass.cuh", "nvfp4pt_dequant.cuh")]
+                            "nvfp4pt_colpass.cuh", "nvfp4pt_dequant.cuh", "nvfp4pt_xform.cuh")]
 # The cast's launches on rows of up to 16384 elements, in order (nvfp4pt_timing.h):
 # zeroing, the row pass, the column pass.
 KERNELS = ("pass0_zero", "rowpass", "colpass")
@@ -511,6 +511,55 @@ def run_gpu_op(args, dist: Dist, op: str) -> dict | None:
     }
 
 
+def run_gpu_opts(args, dist: Dist) -> dict | None:
+    """Device time of nvfp4pt_quantize_grouped_opts (one token group) on the headline
+    activation with the columnwise options: rht (the 16-point transform; its own amax
+    sweep reads x a third time), sr (stochastic rounding, Philox words) or rht_sr."""
+    import torch
+
+    import precision_quantization_row_b200 as nv
+    from precision_quantization_row_b200 import build, inputs
+
+    build.build()
+    torch.cuda.set_device(dist.local_rank)
+    dev = torch.device("cuda", dist.local_rank)
+    stream = torch.cuda.current_stream(dev)
+    m, k = args.rows, args.cols
+    x_host = inputs.llm(M=m, K=k)
+    xs = [x_host.to(dev), x_host.to(dev).clone()]
+    outs = [nv._outputs(m, k, nv.ROWWISE | nv.COLWISE, dev) for _ in range(2)]
+    buf = torch.zeros(1, dtype=torch.float32, device=dev)
+    ws = nv.new_workspace(m, k, device=dev)
+    mode = args.colwise_opts
+    opts = dict(rht="rht" in mode, rht_signs=0xB65C if "rht" in mode else 0, sr="sr" in mode, seed=2024)
+
+    def step(i):
+        nv.quantize_grouped_opts(xs[i & 1], None, absmax=buf, decay=DECAY, out=outs[i & 1], workspace=ws,
+                                 stream=stream, offset=i, **opts)
+
+    secs, all_secs, clocks = timed_regions(args, dist, dev, stream, step)
+    if nv.workspace_error(ws) != 0:
+        raise RuntimeError("device error word set during the timed region")
+    if dist.rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    per = secs / args.steps
+    byts = algo_bytes(m, k) + (2 * m * k if opts["rht"] else 0)   # the transform's amax sweep reads x again
+    achieved = byts / per / 1e9
+    return {
+        "metric": "NVFP4 per-token cast with columnwise options: elems/s, achieved HBM GB/s",
+        "value": float(m) * k * args.steps * dist.world / secs, "unit": "elem/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16->nvfp4", "data": "synthetic",
+        "config": {"workload": f"{workload_name(m, k)}_colwise_{mode}", "rows": m, "cols": k,
+                   "l2": "inputs larger than L2, 2 rotating input copies and output sets"},
+        "timing": region_stats(all_secs),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_kind, "algorithmic_bytes_per_call": byts},
+        "gpu_launches": (nv.CAST_LAUNCHES + (1 if opts["rht"] else 0)) * args.steps, "clocks": clocks,
+    }
+
+
 def measured_tensor_peak():
     """Dense FP4 tensor peak: the measured bf16 burst (cuBLAS) times the nominal FP4/bf16
     ratio 4 (9 and 2.25 PFLOP/s dense), or the fallback bf16 figure times 4."""
@@ -786,6 +835,8 @@ def main(argv=None):
     ap.add_argument("--op", choices=["cast", "dequant", "requant", "gemm"], default="cast",
                     help="cast: the per-token cast (the headline); dequant / requant / gemm: the secondary ops")
     ap.add_argument("--gemm-n", type=int, default=8192, help="N of --op gemm (M = --rows, K = --cols)")
+    ap.add_argument("--colwise-opts", choices=["rht", "sr", "rht_sr"], default=None,
+                    help="time the cast with these columnwise options (the headline activation)")
     ap.add_argument("--config", choices=["llm", "dense", "moe", "weight", "calib"], default="llm",
                     help="llm: the headline activation; the others time the remaining workloads")
     args = ap.parse_args(argv)
@@ -800,6 +851,8 @@ def main(argv=None):
     try:
         if args.config != "llm":
             line = run_gpu_config(args, dist, args.config)
+        elif args.colwise_opts:
+            line = run_gpu_opts(args, dist)
         elif args.op == "gemm":
             line = run_gpu_gemm(args, dist)
         elif args.op != "cast":

@@ -183,6 +183,42 @@ RowShape row_shape(int64_t cols)
     return r;
 }
 
+// One token group, 512-row column tasks: how many of the top row tasks (an even number)
+// to cut into 256-row tasks so that the grid-strided walk (warp w takes tasks T-1-w,
+// T-1-w-W, ..., so the top rows come last) leaves no warp much more work than the mean.
+// Takes the count whose largest per-warp work (in 256-row units) is least, the fewest
+// small tasks on ties. The last shape asked for is remembered.
+int32_t balanced_small_tasks(int64_t rows, int64_t strips, int64_t warps)
+{
+    static std::mutex mu;
+    static int64_t key[3] = {-1, -1, -1};
+    static int32_t val = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (key[0] == rows && key[1] == strips && key[2] == warps) return val;
+    int64_t best_units = INT64_MAX;
+    int32_t best = 0;
+    for (int64_t st = 0; st <= rows / kHalfRows; st += 2) {
+        const int64_t big = (rows - st * kHalfRows + kTaskRows - 1) / kTaskRows;
+        const int64_t T = (st + big) * strips, S = st * strips;   // tasks; the first S are small
+        int64_t worst = 0;
+        for (int64_t w = 0; w < warps && w < T; ++w) {
+            const int64_t n = (T - 1 - w) / warps + 1;        // warp w's tasks: T-1-w-k*warps, k < n
+            const int64_t kfirst = (T - 1 - w >= S) ? (T - 1 - w - S) / warps + 1 : 0;   // first small one
+            const int64_t units = 2 * n - (n > kfirst ? n - kfirst : 0);
+            worst = units > worst ? units : worst;
+        }
+        if (worst < best_units) {
+            best_units = worst;
+            best = (int32_t)st;
+        }
+    }
+    key[0] = rows;
+    key[1] = strips;
+    key[2] = warps;
+    val = best;
+    return val;
+}
+
 template <int MAXG, bool NV>
 cudaError_t launch_rowpass(const RowShape& rs, const RowParams<MAXG>& rp, cudaStream_t stream)
 {
@@ -298,6 +334,15 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
             cp.row_off[g] = (int32_t)off[g];
             cp.task_off[g] = tasks;
             tasks += (int32_t)((off[g + 1] - off[g] + cp.task_rows - 1) / cp.task_rows);
+        }
+        if (MAXG == 1 && cp.task_rows == kTaskRows) {
+            // cut the top row tasks in two where that evens out the warps' work (the
+            // one-group kernel reads small_tasks; the grouped one keeps one task height)
+            const int64_t warps =
+                std::max<int64_t>(1, std::min<int64_t>(dev->sm_count, (tasks * strips + kColWarps - 1) / kColWarps)) *
+                kColWarps;
+            cp.small_tasks = balanced_small_tasks(rows, strips, warps);
+            tasks = cp.small_tasks + (int32_t)((rows - (int64_t)cp.small_tasks * kHalfRows + kTaskRows - 1) / kTaskRows);
         }
         cp.row_off[G] = (int32_t)off[G];
         cp.task_off[G] = tasks;

@@ -42,6 +42,7 @@ struct ColParams {
     int64_t cols;
     int64_t num_tasks;   // row tasks x strips
     int32_t task_rows;   // rows of a task: kTaskRows, or kHalfRows when that leaves warps idle
+    int32_t small_tasks; // one token group: the first small_tasks row tasks have kHalfRows rows
     int32_t strips;      // ceil(cols / 32)
     int32_t num_ctas;
     int32_t num_groups;
@@ -189,9 +190,16 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
         ct.g = g;
         ct.goff = p.row_off[g];
         ct.grows = p.row_off[g + 1] - ct.goff;
-        ct.row0 = ct.goff + (rt - p.task_off[g]) * p.task_rows;
+        int tr = p.task_rows;
+        if (MAXG == 1 && p.small_tasks > 0) {
+            // the top rows (walked last) in 256-row tasks, the rest in 512-row tasks
+            tr = rt < p.small_tasks ? kHalfRows : kTaskRows;
+            ct.row0 = rt < p.small_tasks ? rt * kHalfRows : p.small_tasks * kHalfRows + (rt - p.small_tasks) * kTaskRows;
+        } else {
+            ct.row0 = ct.goff + (rt - p.task_off[g]) * p.task_rows;
+        }
         const int left = ct.goff + ct.grows - ct.row0;
-        ct.nrows = left >= p.task_rows ? p.task_rows : left;
+        ct.nrows = left >= tr ? tr : left;
         ct.c0 = strip * kTaskCols;
     };
     auto step_back = [&]() {
