@@ -366,7 +366,11 @@ uint16_t oracle_f32_to_bf16(float f)
     const uint16_t hi = (uint16_t)(lo + 1);    /* next magnitude away from zero */
     const double a = fabs((double)f);
     const double dl = a - fabs((double)oracle_bf16_to_f32(lo));
-    const double dh = fabs((double)oracle_bf16_to_f32(hi)) - a;
+    /* Above the largest finite bf16 the next magnitude is infinity; IEEE 754's rounding
+     * to nearest treats it as 2^128 (the next step were the exponent range unbounded),
+     * so from halfway to 2^128 upwards the result is infinity. */
+    const double up = ((hi & 0x7FFFu) == 0x7F80u) ? ldexp(1.0, 128) : fabs((double)oracle_bf16_to_f32(hi));
+    const double dh = up - a;
     if (dl < dh) return lo;
     if (dh < dl) return hi;
     return (lo & 1) ? hi : lo;

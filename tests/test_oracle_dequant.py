@@ -21,6 +21,10 @@ def test_bf16_rounding_matches_torch(orc):
         (np.arange(0x3F80, 0x3F80 + 256, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
         -(np.arange(0x0080, 0x0080 + 256, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
         np.array([0.0, -0.0, 1e-45, -1e-45, 3.3e38, -3.3e38], np.float32),
+        # the top of the range: below, at and above halfway from the largest finite bf16
+        # (0x7F7F) to 2^128, where rounding to nearest overflows to infinity
+        np.array([0x7F7F7FFF, 0x7F7F8000, 0x7F7F8001, 0x7F7FFFFF, 0x7F7EFFFF, 0xFF7F8000, 0xFF7F7FFF,
+                  0x7F800000, 0xFF800000], np.uint32).view(np.float32),
     ])
     assert np.array_equal(orc.f32_to_bf16(v), _bf16_bits(torch.from_numpy(v)))
 
