@@ -216,8 +216,8 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w_bf16, int64_
 NVFP4PT_API nvfp4pt_status nvfp4pt_dequantize(const uint8_t* q, const uint8_t* sf, const float* amax,
                                               int64_t rows, int64_t cols, void* out_bf16, cudaStream_t stream);
 
-/* Workspace bytes of nvfp4pt_requantize_colwise: the dequantized bf16 matrix
- * (rows * cols * 2, rounded up to 256) plus nvfp4pt_workspace_bytes(rows, cols, num_groups). */
+/* Workspace bytes of nvfp4pt_requantize_colwise: the rows' fp32 decode scales (rows * 4,
+ * rounded up to 256) plus nvfp4pt_workspace_bytes(rows, cols, num_groups). */
 NVFP4PT_API size_t nvfp4pt_requantize_workspace_bytes(int64_t rows, int64_t cols, int num_groups);
 
 /*

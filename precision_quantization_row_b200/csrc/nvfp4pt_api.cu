@@ -16,6 +16,7 @@
 #include "nvfp4pt_rowpass.cuh"
 #include "nvfp4pt_colpass.cuh"
 #include "nvfp4pt_dequant.cuh"
+#include "nvfp4pt_requant.cuh"
 
 using namespace nvfp4pt;
 
@@ -67,6 +68,12 @@ nvfp4pt_status device_state(DeviceState** out)
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColPass) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
             }
+            const void* rq_tiles[] = {(const void*)rq_tile<1, false>, (const void*)rq_tile<1, true>,
+                                      (const void*)rq_tile<kMaxGroups, false>, (const void*)rq_tile<kMaxGroups, true>};
+            for (const void* f : rq_tiles) {
+                if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemRqTile) != cudaSuccess)
+                    return NVFP4PT_ERR_CUDA;
+            }
             if (!g_encode) {
                 cudaDriverEntryPointQueryResult q;
                 void* fn = nullptr;
@@ -101,6 +108,34 @@ nvfp4pt_status encode_map(CUtensorMap* map, const void* x, int64_t rows, int64_t
     const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+}
+
+// uint8 matrix [rows, width] (row stride `width` bytes, a multiple of 16) in boxes of
+// box_w bytes x box_rows rows, no swizzle; out-of-range bytes read as zero.
+nvfp4pt_status encode_u8_map(CUtensorMap* map, const void* base, int64_t rows, int64_t width, int box_w, int box_rows)
+{
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)width};
+    cuuint32_t box[2] = {(cuuint32_t)box_w, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+}
+
+// fp32 vector [n] as a one-row matrix [1, n], in boxes of `box` elements; out-of-range
+// elements read as zero.
+nvfp4pt_status encode_f32_vector_map(CUtensorMap* map, const float* base, int64_t n, int box)
+{
+    cuuint64_t dims[2] = {(cuuint64_t)n, 1};
+    cuuint64_t strides[1] = {(cuuint64_t)((n * 4 + 15) & ~int64_t(15))};
+    cuuint32_t boxd[2] = {(cuuint32_t)box, 1};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                                boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 
@@ -448,12 +483,89 @@ cudaError_t launch_dequant(const uint8_t* q, const uint8_t* sf, const float* ama
     return cudaGetLastError();
 }
 
-// Requantization scratch ahead of the cast's workspace: the rows' decode scales when the
-// row pass can take the NVFP4 data directly (cols <= kRowPassMaxCols), else the whole
-// dequantized matrix (bf16) for the tile path.
-int64_t requant_scratch_bytes(int64_t rows, int64_t cols)
+// Requantization scratch ahead of the cast's workspace: the rows' decode scales.
+int64_t requant_scratch_bytes(int64_t rows) { return align256(rows * 4); }
+
+// The columnwise requantization (nvfp4pt_requant.cuh): zeroing, rq_colmax, rq_colenc,
+// chained by programmatic dependent launch. ws is a full cast workspace (error word,
+// observed maxima, bf16 column maxima [G, cols]).
+template <int MAXG>
+nvfp4pt_status run_requant(const uint8_t* q, const uint8_t* sf, const float* amax, int64_t rows, int64_t cols,
+                           const int64_t* off, int G, uint8_t* q_col, uint8_t* sf_col, float* amax_col,
+                           float* absmax, float decay, float* dscale, void* ws, cudaStream_t stream)
 {
-    return cols <= kRowPassMaxCols ? align256(rows * 4) : align256(rows * cols * 2);
+    DeviceState* dev = nullptr;
+    const nvfp4pt_status st = device_state(&dev);
+    if (st != NVFP4PT_OK) return st;
+    uint16_t* colmax = ws_colmax(ws, G);
+    ZeroParams z;
+    std::memset(&z, 0, sizeof z);
+    z.ptr[1] = reinterpret_cast<float4*>(amax_col);
+    z.n4[1] = (int64_t)G * cols / 4;
+    if (absmax) {
+        z.ptr[2] = reinterpret_cast<float4*>(ws_obs(ws));
+        z.n4[2] = pad4(G) / 4;
+    }
+    z.ptr[3] = reinterpret_cast<float4*>(colmax);
+    z.n4[3] = (int64_t)G * cols * 2 / 16;
+    z.err = ws_err(ws);
+    if (launch_zero(stream, z) != cudaSuccess) return NVFP4PT_ERR_CUDA;
+
+    RqParams<MAXG> p;
+    std::memset(&p, 0, sizeof p);
+    p.q = q;
+    p.sf = sf;
+    p.amax = amax;
+    p.dscale = dscale;
+    p.colmax = colmax;
+    p.obs = absmax ? ws_obs(ws) : nullptr;
+    p.q_col = q_col;
+    p.sf_col = sf_col;
+    p.amax_col = amax_col;
+    p.absmax = absmax;
+    p.decay = decay;
+    p.nbuf = absmax ? G : 0;
+    p.rows = rows;
+    p.cols = cols;
+    p.chunks = (cols + kRqChunkCols - 1) / kRqChunkCols;
+    p.slices = rows / kRqSliceRows;
+    p.strips = (int32_t)((cols + kRqStripCols - 1) / kRqStripCols);
+    p.num_groups = G;
+    int64_t steps = 0;
+    for (int g = 0; g < G; ++g) {
+        p.row_off[g] = (int32_t)off[g];
+        p.step_off[g] = (int32_t)steps;
+        steps += (off[g + 1] - off[g] + kRqStepRows - 1) / kRqStepRows;
+    }
+    p.row_off[G] = (int32_t)rows;
+    p.step_off[G] = (int32_t)steps;
+    const int64_t sms = dev->sm_count;
+    if (cols % kRtCols == 0) {
+        // whole 256-column tiles: the TMA-fed kernels
+        int64_t tsteps = 0;
+        for (int g = 0; g < G; ++g) {
+            p.tstep_off[g] = (int32_t)tsteps;
+            tsteps += (off[g + 1] - off[g] + kRtRows - 1) / kRtRows;
+        }
+        p.tstep_off[G] = (int32_t)tsteps;
+        p.err = ws_err(ws);
+        if (encode_u8_map(&p.tm_q, q, rows, cols / 2, kRtCols / 2, kRtRows) != NVFP4PT_OK ||
+            encode_u8_map(&p.tm_sf, sf, rows, cols / 16, kRtCols / 16, kRtRows) != NVFP4PT_OK ||
+            encode_f32_vector_map(&p.tm_amax, amax, rows, kRtRows) != NVFP4PT_OK)
+            return NVFP4PT_ERR_CUDA;
+        const int grid = (int)std::min<int64_t>((cols / kRtCols) * tsteps, 2 * sms);
+        if (launch(rq_tile<MAXG, false>, grid, kSmemRqTile, stream, p, true, kRtThreads) != cudaSuccess ||
+            launch(rq_tile<MAXG, true>, grid, kSmemRqTile, stream, p, true, kRtThreads) != cudaSuccess)
+            return NVFP4PT_ERR_CUDA;
+        return NVFP4PT_OK;
+    }
+    const int64_t warps1 = p.slices * p.chunks, warps2 = steps * p.strips;
+    const int grid1 = (int)std::min<int64_t>((warps1 + kRqWarps - 1) / kRqWarps, 3 * sms);
+    const int grid2 = (int)std::min<int64_t>((warps2 + kRqWarps - 1) / kRqWarps, 2 * sms);
+    if (launch(rq_colmax<MAXG>, grid1, 0, stream, p, true, kRqThreads) != cudaSuccess ||
+        launch(rq_colenc<MAXG>, grid2, 0, stream, p, true, kRqThreads) != cudaSuccess)
+        return NVFP4PT_ERR_CUDA;
+    return NVFP4PT_OK;
 }
 
 }  // namespace
@@ -653,8 +765,7 @@ nvfp4pt_status nvfp4pt_dequantize(const uint8_t* q, const uint8_t* sf, const flo
 
 size_t nvfp4pt_requantize_workspace_bytes(int64_t rows, int64_t cols, int num_groups)
 {
-    const int64_t r = rows < 0 ? 0 : rows, c = cols < 0 ? 0 : cols;
-    return (size_t)requant_scratch_bytes(r, c) + nvfp4pt_workspace_bytes(rows, cols, num_groups);
+    return (size_t)requant_scratch_bytes(rows < 0 ? 0 : rows) + nvfp4pt_workspace_bytes(rows, cols, num_groups);
 }
 
 nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, const uint8_t* sf_row, const float* amax_row,
@@ -676,25 +787,13 @@ nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, const uint8_t* s
         if (off[g + 1] < off[g] || off[g] % 16) return NVFP4PT_ERR_GROUPS;
     DeviceState* dev = nullptr;
     if ((st = device_state(&dev)) != NVFP4PT_OK) return st;
-    void* ws = static_cast<uint8_t*>(workspace) + requant_scratch_bytes(rows, cols);
-    if (cols <= kRowPassMaxCols) {
-        // the row pass and the column pass read the NVFP4 data themselves
-        const NvSource src{q_row, sf_row, amax_row, static_cast<float*>(workspace)};
-        if (G == 1)
-            return run_cast<1>(nullptr, rows, cols, off, 1, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col,
-                               sf_col, amax_col, absmax_bufs, decay, false, ws, stream, nullptr, true, &src);
-        return run_cast<kMaxGroups>(nullptr, rows, cols, off, G, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col,
-                                    sf_col, amax_col, absmax_bufs, decay, false, ws, stream, nullptr, true, &src);
-    }
-    // X' (bf16) in the workspace, then the columnwise cast of X' with the rest of it
-    uint16_t* xd = static_cast<uint16_t*>(workspace);
-    if (launch_dequant(q_row, sf_row, amax_row, rows, cols, xd, dev->sm_count, stream) != cudaSuccess)
-        return NVFP4PT_ERR_CUDA;
+    float* dscale = static_cast<float*>(workspace);
+    void* ws = static_cast<uint8_t*>(workspace) + requant_scratch_bytes(rows);
     if (G == 1)
-        return run_cast<1>(xd, rows, cols, off, 1, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col, sf_col,
-                           amax_col, absmax_bufs, decay, false, ws, stream);
-    return run_cast<kMaxGroups>(xd, rows, cols, off, G, NVFP4PT_COLWISE, nullptr, nullptr, nullptr, q_col, sf_col,
-                                amax_col, absmax_bufs, decay, false, ws, stream);
+        return run_requant<1>(q_row, sf_row, amax_row, rows, cols, off, 1, q_col, sf_col, amax_col, absmax_bufs,
+                              decay, dscale, ws, stream);
+    return run_requant<kMaxGroups>(q_row, sf_row, amax_row, rows, cols, off, G, q_col, sf_col, amax_col,
+                                   absmax_bufs, decay, dscale, ws, stream);
 }
 
 }  // extern "C"

@@ -148,10 +148,11 @@ def test_dequant_and_requant_rejections(L):
     assert d(P(), P(), P(), 16, 24, P(), None) == 2
     assert d(P(), P(8), P(), 16, 16, P(), None) == 3
     assert d(P(), P(), P(), 16, 16, P(4), None) == 3
-    # the rows' decode scales (cols <= 16384), else the dequantized bf16 matrix
-    assert L.nvfp4pt_requantize_workspace_bytes(16, 16, 1) >= 16 * 4 + L.nvfp4pt_workspace_bytes(16, 16, 1)
-    assert (L.nvfp4pt_requantize_workspace_bytes(16, 16400, 1) >=
-            16 * 16400 * 2 + L.nvfp4pt_workspace_bytes(16, 16400, 1))
+    # the rows' decode scales, then a cast workspace, at any width
+    for cols in (16, 16400):
+        assert (L.nvfp4pt_requantize_workspace_bytes(16, cols, 1) ==
+                256 + L.nvfp4pt_workspace_bytes(16, cols, 1))
+    assert L.nvfp4pt_requantize_workspace_bytes(1024, 64, 3) == 4096 + L.nvfp4pt_workspace_bytes(1024, 64, 3)
 
     def r(*args, offs=None, G=1, rows=64, ws=None):
         arr = None if offs is None else (ctypes.c_int64 * len(offs))(*offs)

@@ -35,6 +35,20 @@ def test_dequant_random_codes(orc, shape):
     assert bad.size == 0, f"{bad.shape[0]} mismatches, first {bad[:3].tolist()}"
 
 
+def test_dequant_overflows_to_infinity(orc):
+    """Row amaxes up to the largest binary32: products at or past halfway from the largest
+    finite bf16 to 2^128 round to infinity, below it to the largest finite bf16."""
+    rng = np.random.default_rng(68)
+    rows, cols = 64, 128
+    q = rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
+    sf = rng.choice([0x7E, 0x7D, 0x76, 0x70, 0xFE], (rows, cols // 16)).astype(np.uint8)
+    amax = np.linspace(3.0e38, np.finfo(np.float32).max, rows).astype(np.float32)
+    want = orc.dequantize(q, sf, amax)
+    assert (want & 0x7FFF == 0x7F80).any() and (want & 0x7FFF == 0x7F7F).any()
+    got = nv.dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(), torch.from_numpy(amax).cuda())
+    assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
 @pytest.mark.parametrize("shape", [(272, 1056), (48, 80)], ids=lambda s: f"{s[0]}x{s[1]}")
 def test_dequant_output_16_byte_aligned(orc, shape):
     """An output 16 bytes past a 32-byte boundary: each block goes out as two 16-byte
@@ -75,8 +89,8 @@ def _rows_of(x):
     return out["q_row"], out["sf_row"], out["amax_row"]
 
 
-# (64, 12288): two blocks per row-pass thread; (64, 16400): rows wider than 16384 take
-# the dequantize-then-cast route
+# (48, 80): a 64-column strip with a partial 8-column group and a 16-row step;
+# (64, 16400): rows wider than the cast's row pass takes
 @pytest.mark.parametrize("shape", [(256, 512), (1040, 1056), (4096, 4096), (48, 80), (64, 12288), (64, 16400)],
                          ids=lambda s: f"{s[0]}x{s[1]}")
 def test_requant_colwise(orc, shape):
@@ -103,13 +117,48 @@ def test_requant_grouped(orc):
 
 
 def test_requant_grouped_wide_rows(orc):
-    """Grouped requantization of rows 12288 wide (two blocks per row-pass thread)."""
+    """Grouped requantization of rows 12288 wide."""
     x = inputs.random_shape(65, 128, 12288, "normal")
     offsets = [0, 64, 64, 128]
     q, sf, a = _rows_of(x)
     got = nv.requantize_colwise(q, sf, a, offsets=offsets)
     want = orc.requantize_colwise(q.cpu().numpy(), sf.cpu().numpy(), a.cpu().numpy(), offsets=offsets)
     compare(to_np(got), {k: want[k] for k in ("q_col", "sf_col", "amax_col")}, label="grouped requant wide")
+
+
+# widths that are multiples of 256 take the TMA-fed tile kernels, the others the direct ones
+@pytest.mark.parametrize("shape,offsets", [((48, 80), None), ((272, 144), None), ((96, 4112), None),
+                                          ((400, 272), [0, 16, 16, 240, 400]), ((528, 336), [0, 0, 512, 528]),
+                                          ((304, 512), None), ((400, 768), [0, 16, 16, 240, 400]),
+                                          ((176, 1280), [0, 0, 48, 112, 176, 176])],
+                         ids=["48x80", "272x144", "96x4112", "400x272g", "528x336g", "304x512", "400x768g",
+                              "176x1280g"])
+def test_requant_random_codes(orc, shape, offsets):
+    """Arbitrary codes, every finite block-scale code (negative and subnormal ones too) and
+    extreme row amaxes: the requantization is the oracle's columnwise cast of the oracle's
+    dequantization, codes, scales, column amaxes and running buffers."""
+    q, sf, amax = _random_rows(sum(shape) + 7, *shape)
+    G = 1 if offsets is None else len(offsets) - 1
+    bufs = torch.linspace(0.5, 4.0, G, dtype=torch.float32, device="cuda")
+    want = orc.requantize_colwise(q, sf, amax, offsets=offsets, absmax=bufs.cpu().numpy(), decay=0.5)
+    got = nv.requantize_colwise(torch.from_numpy(q).cuda(), torch.from_numpy(sf).cuda(),
+                                torch.from_numpy(amax).cuda(), offsets=offsets, absmax=bufs, decay=0.5)
+    compare(to_np(got), {k: want[k] for k in ("q_col", "sf_col", "amax_col")}, label=f"requant random {shape}")
+    assert np.array_equal(bufs.cpu().numpy().view(np.uint32), want["absmax"].view(np.uint32))
+
+
+@pytest.mark.parametrize("cols", [64, 256])
+def test_requant_many_groups(orc, cols):
+    """1024 token groups of 16 rows (and some empty ones): one 16-row step per group."""
+    rows = 16 * 1000
+    x = inputs.random_shape(66, rows, cols, "normal")
+    sizes = [16] * 1000 + [0] * 24
+    np.random.default_rng(67).shuffle(sizes)
+    offsets = [0] + list(np.cumsum(sizes))
+    q, sf, a = _rows_of(x)
+    got = nv.requantize_colwise(q, sf, a, offsets=offsets)
+    want = orc.requantize_colwise(q.cpu().numpy(), sf.cpu().numpy(), a.cpu().numpy(), offsets=offsets)
+    compare(to_np(got), {k: want[k] for k in ("q_col", "sf_col", "amax_col")}, label="requant 1024 groups")
 
 
 def test_requant_of_lossless_rows_equals_direct_cast():
