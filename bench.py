@@ -46,7 +46,8 @@ def workload_name(m: int, k: int) -> str:
 PROFILE_JSON = os.path.join(ROOT, "profiles", "nvfp4pt_cast_llm_16384x8192.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "precision_quantization_row_b200", "csrc", f)
                   for f in ("nvfp4pt_api.cu", "nvfp4pt_device.cuh", "nvfp4pt_kernels.cuh", "nvfp4pt_rowpass.cuh",
-                            "nvfp4pt_colpass.cuh", "nvfp4pt_dequant.cuh", "nvfp4pt_xform.cuh")]
+                            "nvfp4pt_colpass.cuh", "nvfp4pt_colpass_tma.cuh", "nvfp4pt_dequant.cuh",
+                            "nvfp4pt_xform.cuh")]
 # The cast's launches on rows of up to 16384 elements, in order (nvfp4pt_timing.h):
 # zeroing, the row pass, the column pass.
 KERNELS = ("pass0_zero", "rowpass", "colpass")

@@ -15,6 +15,7 @@
 #include "nvfp4pt_kernels.cuh"
 #include "nvfp4pt_rowpass.cuh"
 #include "nvfp4pt_colpass.cuh"
+#include "nvfp4pt_colpass_tma.cuh"
 #include "nvfp4pt_dequant.cuh"
 #include "nvfp4pt_requant.cuh"
 
@@ -68,6 +69,19 @@ nvfp4pt_status device_state(DeviceState** out)
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColPass) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
             }
+            const void* tcols[] = {(const void*)colpass_tma<1>, (const void*)colpass_tma<kMaxGroups>};
+            for (const void* f : tcols) {
+                if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColTma) != cudaSuccess ||
+                    cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+                    return NVFP4PT_ERR_CUDA;
+            }
+            // the one-group row passes use a few KB of shared memory: the rest of the SM's
+            // on-chip memory is theirs as L1
+            const void* rps[] = {(const void*)rowpass<1, 1, 4, false>, (const void*)rowpass<1, 2, 2, false>,
+                                 (const void*)rowpass<1, 1, 2, false>, (const void*)rowpass<1, 1, 1, false>};
+            for (const void* f : rps)
+                if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 0) != cudaSuccess)
+                    return NVFP4PT_ERR_CUDA;
             const void* rq_tiles[] = {(const void*)rq_tile<1, false>, (const void*)rq_tile<1, true>,
                                       (const void*)rq_tile<kMaxGroups, false>, (const void*)rq_tile<kMaxGroups, true>};
             for (const void* f : rq_tiles) {
@@ -362,8 +376,13 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
             for (int g = 0; g < G; ++g) t += (off[g + 1] - off[g] + tr - 1) / tr;
             return t;
         };
-        cp.task_rows = count_tasks(kTaskRows) * strips >= 2 * (int64_t)dev->sm_count * kColWarps ? kTaskRows
-                                                                                                 : kHalfRows;
+        // The plain encode of one token group with at least four 512-row tasks per warp runs
+        // colpass_tma (kTcWarps warps per CTA); smaller or grouped casts and the options
+        // run colpass, whose 16 warps per CTA even out fewer tasks.
+        const int64_t tasks512 = count_tasks(kTaskRows) * strips;
+        const bool tma_col = !opts && !nv && MAXG == 1 && tasks512 >= 4 * (int64_t)dev->sm_count * kTcWarps;
+        const int64_t cw = tma_col ? kTcWarps : kColWarps;
+        cp.task_rows = tasks512 >= 2 * (int64_t)dev->sm_count * cw ? kTaskRows : kHalfRows;
         int32_t tasks = 0;
         for (int g = 0; g < G; ++g) {
             cp.row_off[g] = (int32_t)off[g];
@@ -374,8 +393,7 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
             // cut the top row tasks in two where that evens out the warps' work (the
             // one-group kernel reads small_tasks; the grouped one keeps one task height)
             const int64_t warps =
-                std::max<int64_t>(1, std::min<int64_t>(dev->sm_count, (tasks * strips + kColWarps - 1) / kColWarps)) *
-                kColWarps;
+                std::max<int64_t>(1, std::min<int64_t>(dev->sm_count, (tasks * strips + cw - 1) / cw)) * cw;
             cp.small_tasks = balanced_small_tasks(rows, strips, warps);
             tasks = cp.small_tasks + (int32_t)((rows - (int64_t)cp.small_tasks * kHalfRows + kTaskRows - 1) / kTaskRows);
         }
@@ -406,6 +424,25 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         cp.sf_col = sf_col;
         cp.absmax = absmax;
         cp.obs = ws_obs(ws);
+        cp.err = ws_err(ws);
+        if (tma_col) {
+            // steps copied by TMA (boxes of 32 columns x 64 rows of x)
+            ColTmaParams<MAXG> tp;
+            std::memset(&tp, 0, sizeof tp);
+            tp.c = cp;
+            tp.c.num_ctas = (int32_t)std::max<int64_t>(
+                1, std::min<int64_t>(dev->sm_count, (cp.num_tasks + kTcWarps - 1) / kTcWarps));
+            cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+            cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+            cuuint32_t box[2] = {(cuuint32_t)kTaskCols, (cuuint32_t)kStepRows};
+            cuuint32_t estr[2] = {1, 1};
+            if (g_encode(&tp.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return NVFP4PT_ERR_CUDA;
+            e = launch(colpass_tma<MAXG>, tp.c.num_ctas, kSmemColTma, stream, tp, true, kTcThreads);
+            return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+        }
         if (opts) {
             cp.rht = co->rht;
             cp.rht_signs = co->rht_signs & 0xFFFFu;

@@ -65,6 +65,7 @@ struct ColParams {
     uint8_t* sf_col;
     float* absmax;           // [nbuf] running amax buffers, or null
     const float* obs;        // [G] amax observed by the row pass
+    uint32_t* err;           // device error word (colpass_tma: a copy that never landed)
     // columnwise options (nvfp4pt_xform.cuh): the Hadamard transform with its sign mask,
     // stochastic rounding with its Philox key and counter offset
     int32_t rht;

@@ -63,6 +63,19 @@ def test_llm_config_full(orc):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("flags", [RC, nv.COLWISE], ids=["rowcol", "colwise"])
+def test_large_ragged_cast(orc, flags):
+    """10000 x 7600: enough 512-row x 32-column tasks (4760) for the TMA-fed column pass,
+    with ragged row tasks (10000 = 19 x 512 + 272) and a half-width last column strip."""
+    x = inputs.random_shape(70, 10000, 7600, "wide")
+    got = gpu_cast(x, flags=flags, absmax=3.0, decay=0.5)
+    want = oracle_quantize_parallel(x, flags=flags)
+    compare({k: got[k] for k in want if k != "amax_row" or flags & nv.ROWWISE}, want, label="large ragged",
+            keys=[k for k in want if k != "amax_row" or flags & nv.ROWWISE])
+    assert got["absmax"][0] == max(np.float32(1.5), want["amax_col"].max())
+
+
+@pytest.mark.slow
 def test_moe_grouped_config_full(orc):
     x, offsets = inputs.moe()
     G = len(offsets) - 1
