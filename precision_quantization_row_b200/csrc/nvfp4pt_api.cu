@@ -61,10 +61,8 @@ nvfp4pt_status device_state(DeviceState** out)
                     cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
             }
-            const void* colpasses[] = {(const void*)colpass<1, false>, (const void*)colpass<kMaxGroups, false>,
-                                       (const void*)colpass<1, true>, (const void*)colpass<kMaxGroups, true>,
-                                       (const void*)colpass<1, false, kColOpts>,
-                                       (const void*)colpass<kMaxGroups, false, kColOpts>};
+            const void* colpasses[] = {(const void*)colpass<1>, (const void*)colpass<kMaxGroups>,
+                                       (const void*)colpass<1, kColOpts>, (const void*)colpass<kMaxGroups, kColOpts>};
             for (const void* f : colpasses) {
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemColPass) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
@@ -77,8 +75,8 @@ nvfp4pt_status device_state(DeviceState** out)
             }
             // the one-group row passes use a few KB of shared memory: the rest of the SM's
             // on-chip memory is theirs as L1
-            const void* rps[] = {(const void*)rowpass<1, 1, 4, false>, (const void*)rowpass<1, 2, 2, false>,
-                                 (const void*)rowpass<1, 1, 2, false>, (const void*)rowpass<1, 1, 1, false>};
+            const void* rps[] = {(const void*)rowpass<1, 1, 4>, (const void*)rowpass<1, 2, 2>, (const void*)rowpass<1, 1, 2>,
+                                 (const void*)rowpass<1, 1, 1>};
             for (const void* f : rps)
                 if (cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 0) != cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
@@ -268,14 +266,14 @@ int32_t balanced_small_tasks(int64_t rows, int64_t strips, int64_t warps)
     return val;
 }
 
-template <int MAXG, bool NV>
+template <int MAXG>
 cudaError_t launch_rowpass(const RowShape& rs, const RowParams<MAXG>& rp, cudaStream_t stream)
 {
     const int grid = rp.num_ctas;
-    if (rs.bt == 2) return launch(rowpass<MAXG, 2, 2, NV>, grid, 0, stream, rp, true, kRowThreads);
-    if (rs.S == 4) return launch(rowpass<MAXG, 1, 4, NV>, grid, 0, stream, rp, true, kRowThreads);
-    if (rs.S == 2) return launch(rowpass<MAXG, 1, 2, NV>, grid, 0, stream, rp, true, kRowThreads);
-    return launch(rowpass<MAXG, 1, 1, NV>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.bt == 2) return launch(rowpass<MAXG, 2, 2>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.S == 4) return launch(rowpass<MAXG, 1, 4>, grid, 0, stream, rp, true, kRowThreads);
+    if (rs.S == 2) return launch(rowpass<MAXG, 1, 2>, grid, 0, stream, rp, true, kRowThreads);
+    return launch(rowpass<MAXG, 1, 1>, grid, 0, stream, rp, true, kRowThreads);
 }
 
 // The columnwise options of a call (nvfp4pt_colwise_options), as the kernels take them.
@@ -287,21 +285,11 @@ struct ColOptions {
     uint64_t offset;
 };
 
-// NVFP4 rowwise data as the cast's source (the requantization): codes, scales, row
-// amaxes, and room for the rows' decode scales.
-struct NvSource {
-    const uint8_t* q;
-    const uint8_t* sf;
-    const float* amax;
-    float* dscale;
-};
-
 template <int MAXG>
 nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t* off, int G, int flags,
                         uint8_t* q_row, uint8_t* sf_row, float* amax_row, uint8_t* q_col, uint8_t* sf_col,
                         float* amax_col, float* absmax, float decay, bool w2d, void* ws, cudaStream_t stream,
-                        void* const* events = nullptr, bool full_ws = true, const NvSource* nv = nullptr,
-                        const ColOptions* co = nullptr)
+                        void* const* events = nullptr, bool full_ws = true, const ColOptions* co = nullptr)
 {
     // events[0] before the first launch, events[i] after the i-th (measurement hook)
     auto mark = [&](int i) -> bool {
@@ -347,21 +335,14 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         rp.do_row = do_row;
         rp.strided = G == 1;
         rp.x = static_cast<const uint16_t*>(x);
-        if (nv) {
-            rp.nq = nv->q;
-            rp.nsf = nv->sf;
-            rp.namax = nv->amax;
-            rp.dscale = nv->dscale;
-            rp.do_row = 0;
-        }
-        rp.amax_row = (do_row && !nv) ? amax_row : nullptr;
+        rp.amax_row = do_row ? amax_row : nullptr;
         rp.q_row = q_row;
         rp.sf_row = sf_row;
         rp.amax_col = (do_col && !colmax && !xf_amax) ? amax_col : nullptr;
         rp.colmax = reinterpret_cast<uint32_t*>(colmax);
         rp.obs = absmax ? ws_obs(ws) : nullptr;
         for (int g = 0; g <= G; ++g) rp.row_off[g] = (int32_t)off[g];
-        e = nv ? launch_rowpass<MAXG, true>(rs, rp, stream) : launch_rowpass<MAXG, false>(rs, rp, stream);
+        e = launch_rowpass<MAXG>(rs, rp, stream);
         if (e != cudaSuccess || !mark(2)) return NVFP4PT_ERR_CUDA;
 
         // Column pass: 256-row tasks per group (the last one ragged) x 32-column strips.
@@ -380,7 +361,7 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         // colpass_tma (kTcWarps warps per CTA); smaller or grouped casts and the options
         // run colpass, whose 16 warps per CTA even out fewer tasks.
         const int64_t tasks512 = count_tasks(kTaskRows) * strips;
-        const bool tma_col = !opts && !nv && MAXG == 1 && tasks512 >= 4 * (int64_t)dev->sm_count * kTcWarps;
+        const bool tma_col = !opts && MAXG == 1 && tasks512 >= 4 * (int64_t)dev->sm_count * kTcWarps;
         const int64_t cw = tma_col ? kTcWarps : kColWarps;
         cp.task_rows = tasks512 >= 2 * (int64_t)dev->sm_count * cw ? kTaskRows : kHalfRows;
         int32_t tasks = 0;
@@ -413,11 +394,6 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
         cp.back_rt = (int32_t)(wstride / cp.strips);
         cp.back_strip = (int32_t)(wstride % cp.strips);
         cp.x = static_cast<const uint16_t*>(x);
-        if (nv) {
-            cp.nq = nv->q;
-            cp.nsf = nv->sf;
-            cp.dscale = nv->dscale;
-        }
         cp.amax_col = amax_col;
         cp.colmax = colmax;
         cp.q_col = q_col;
@@ -455,15 +431,14 @@ nvfp4pt_status run_cast(const void* x, int64_t rows, int64_t cols, const int64_t
                 ColParams<MAXG> ap = cp;
                 ap.absmax = nullptr;
                 ap.nbuf = 0;
-                if (launch(colpass<MAXG, false, kColXformAmax>, ap.num_ctas, 0, stream, ap, true, kColThreads) !=
+                if (launch(colpass<MAXG, kColXformAmax>, ap.num_ctas, 0, stream, ap, true, kColThreads) !=
                     cudaSuccess)
                     return NVFP4PT_ERR_CUDA;
             }
-            e = launch(colpass<MAXG, false, kColOpts>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
+            e = launch(colpass<MAXG, kColOpts>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
             return e == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
         }
-        e = nv ? launch(colpass<MAXG, true>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads)
-               : launch(colpass<MAXG, false>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
+        e = launch(colpass<MAXG>, cp.num_ctas, kSmemColPass, stream, cp, true, kColThreads);
         return e == cudaSuccess && mark(3) ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
     }
 
@@ -745,7 +720,7 @@ nvfp4pt_status nvfp4pt_quantize_grouped_opts(const void* x, int64_t rows, int64_
         if ((co.rht || co.sr) && (flags & NVFP4PT_COLWISE) && cols > kRowPassMaxCols) return NVFP4PT_ERR_SHAPE;
     }
     return run_cast<kMaxGroups>(x, rows, cols, offsets, num_groups, flags, q_row, sf_row, amax_row, q_col, sf_col,
-                                amax_col, absmax_bufs, decay, false, workspace, stream, nullptr, true, nullptr, &co);
+                                amax_col, absmax_bufs, decay, false, workspace, stream, nullptr, true, &co);
 }
 
 nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w, int64_t rows, int64_t cols, uint8_t* q_row,

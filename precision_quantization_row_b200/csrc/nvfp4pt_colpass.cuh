@@ -23,7 +23,7 @@
 // every 16th from its end, which lines up with the contiguous runs of the row pass.
 #pragma once
 
-#include "nvfp4pt_dequant.cuh"
+#include "nvfp4pt_device.cuh"
 #include "nvfp4pt_xform.cuh"
 
 namespace nvfp4pt {
@@ -53,11 +53,6 @@ struct ColParams {
     int32_t back_rt;     // a warp's next task is wstride tasks back:
     int32_t back_strip;  //   wstride = back_rt * strips + back_strip, back_strip < strips
     const uint16_t* x;
-    // NVFP4 rowwise source instead of x (the requantization): codes [rows, cols/2],
-    // scales [rows, cols/16] and the rows' decode scales (left by the row pass)
-    const uint8_t* nq;
-    const uint8_t* nsf;
-    const float* dscale;
     float* amax_col;         // [G, cols] fp32: final when the row pass has ended, or (when colmax is
                              //   set) written here from colmax
     const uint16_t* colmax;  // [G, cols] bf16 column maxima left by the row pass, or null
@@ -149,9 +144,8 @@ __device__ __forceinline__ int group_of_task(const ColParams<MAXG>& p, int rt)
     return lo;
 }
 
-// NV = false: x is bf16. NV = true: the rows come dequantized from NVFP4 rowwise data
-// (nq, nsf, dscale), to the same bf16 values nvfp4pt_dequantize gives. MODE: ColMode.
-template <int MAXG, bool NV = false, int MODE = kColPlain>
+// MODE: ColMode.
+template <int MAXG, int MODE = kColPlain>
 __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant__ ColParams<MAXG> p)
 {
     // per warp: codes [column][16 chunks of 8 bytes] (swizzled), then scales [column][32]
@@ -217,30 +211,18 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
         const int c = ct.c0 + 4 * quad;
         const int r = kStepRows * step + 16 * blk;
         const bool ok = r < ct.nrows && c < cols;
-        if constexpr (NV) {
-            // raw: the four columns' 2 code bytes and the block's scale byte per row
-            const int64_t row = ct.row0 + r;
-            const uint16_t* qs = reinterpret_cast<const uint16_t*>(p.nq + row * (cols / 2) + c / 2);
-            const uint8_t* ss = p.nsf + row * (cols / 16) + c / 16;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x + (int64_t)(ct.row0 + r) * cols + c);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                v[i][0] = ok ? (uint32_t)__ldg(qs + i * (cols / 4)) : 0u;
-                v[i][1] = ok ? (uint32_t)__ldg(ss + i * (cols / 16)) : 0u;
+        for (int i = 0; i < 16; ++i) {
+            if (ok) {
+                const uint2 w = ldg_stream64(src);
+                v[i][0] = w.x;
+                v[i][1] = w.y;
+            } else {
+                v[i][0] = 0u;
+                v[i][1] = 0u;
             }
-        } else {
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(p.x + (int64_t)(ct.row0 + r) * cols + c);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                if (ok) {
-                    const uint2 w = ldg_stream64(src);
-                    v[i][0] = w.x;
-                    v[i][1] = w.y;
-                } else {
-                    v[i][0] = 0u;
-                    v[i][1] = 0u;
-                }
-                src += row_bytes;
-            }
+            src += row_bytes;
         }
     };
     // amax of column 4q + j of a task for lane 4q + j (g is the task's group)
@@ -321,24 +303,6 @@ __global__ void __launch_bounds__(kColThreads, 1) colpass(const __grid_constant_
         }
         if (more) load(nxt, nstep, vn);
 
-        if constexpr (NV) {
-            // dequantize this step's raw rows in place, with the rows' decode scales
-            const int r = kStepRows * step + 16 * blk;
-            if (r < cur.nrows && cur.c0 + 4 * quad < cols) {
-                const float4* ds = reinterpret_cast<const float4*>(p.dscale + cur.row0 + r);
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const float4 d = __ldg(ds + i4);
-                    const float m4[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-                    for (int i = 4 * i4; i < 4 * i4 + 4; ++i) {
-                        float sv, s_unused;
-                        e4m3x2_decode(v[i][1], sv, s_unused);
-                        dequant4(v[i][0], sv, m4[i - 4 * i4], v[i][0], v[i][1]);
-                    }
-                }
-            }
-        }
 
         if constexpr (MODE == kColPlain) {
             // block amax of the four columns over this lane's 16 rows

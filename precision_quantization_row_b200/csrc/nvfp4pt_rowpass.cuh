@@ -21,7 +21,7 @@
 // go out to amax_col) about once per group rather than once per batch.
 #pragma once
 
-#include "nvfp4pt_dequant.cuh"
+#include "nvfp4pt_device.cuh"
 
 namespace nvfp4pt {
 
@@ -40,13 +40,6 @@ struct RowParams {
     int32_t do_row;      // write rowwise codes and scales
     int32_t strided;     // batches c, c + num_ctas, ... (else a contiguous run per CTA)
     const uint16_t* x;
-    // NVFP4 rowwise source instead of x (the requantization): codes [rows, cols/2],
-    // scales [rows, cols/16], amaxes [rows]; dscale [rows] receives each row's decode
-    // scale RN(amax / 2688)
-    const uint8_t* nq;
-    const uint8_t* nsf;
-    const float* namax;
-    float* dscale;
     float* amax_row;     // [rows], written directly (not accumulated)
     uint8_t* q_row;
     uint8_t* sf_row;
@@ -82,10 +75,7 @@ __device__ __forceinline__ void encode_block_pair(const uint32_t (&a)[8], const 
     qb1 = encode8(b[4], b[5], b[6], b[7], eb);
 }
 
-// NV = false: x is bf16. NV = true: the rows are dequantized from NVFP4 rowwise data
-// (nq, nsf, namax) as they arrive, to the same bf16 values nvfp4pt_dequantize gives;
-// nothing rowwise is written then.
-template <int MAXG, int BT, int S, bool NV = false>
+template <int MAXG, int BT, int S>
 __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant__ RowParams<MAXG> p)
 {
     griddep_launch_dependents();
@@ -135,14 +125,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
             const int64_t row = r0 + s * p.rps + rsw;
 #pragma unroll
             for (int b = 0; b < BT; ++b) {
-                if (valid[b] && NV) {
-                    // raw block: 8 code bytes, the scale byte, the row's amax bits
-                    const uint2 c8 = ldg_stream64(p.nq + row * (cols / 2) + 8 * (int64_t)bj[b]);
-                    v[s][b][0] = c8.x;
-                    v[s][b][1] = c8.y;
-                    v[s][b][2] = p.nsf[row * (cols / 16) + bj[b]];
-                    v[s][b][3] = __float_as_uint(p.namax[row]);
-                } else if (valid[b]) {
+                if (valid[b]) {
                     ldg256_stream(p.x + row * cols + 16 * (int64_t)bj[b], v[s][b]);
                 } else {
 #pragma unroll
@@ -195,22 +178,9 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
     };
 
     int g_cur = group_of_row(p, b0 * rows_per_batch);
-    auto process = [&](int64_t batch, bool more, uint32_t (&raw)[S][BT][8], uint32_t (&nxt)[S][BT][8]) {
+    auto process = [&](int64_t batch, bool more, uint32_t (&cur)[S][BT][8], uint32_t (&nxt)[S][BT][8]) {
         if (more) load(batch + bstep, nxt);
         const int64_t r0 = batch * rows_per_batch;
-        // the batch's rows as bf16 words: as loaded, or dequantized from the raw blocks
-        uint32_t deq[S][BT][8];
-        if constexpr (NV) {
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                const float m = __fdiv_rn(__uint_as_float(raw[s][0][3]), 2688.0f);   // decode scale of the row
-#pragma unroll
-                for (int b = 0; b < BT; ++b)
-                    dequant16(make_uint2(raw[s][b][0], raw[s][b][1]), raw[s][b][2], m, deq[s][b]);
-                if (p.dscale && tj == 0 && active) p.dscale[r0 + s * p.rps + rsw] = m;
-            }
-        }
-        uint32_t (&cur)[S][BT][8] = NV ? deq : raw;
 
         // block amaxes (kept for the encode), row partials (one per warp and row),
         // column partials
@@ -246,7 +216,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) rowpass(const __grid_constant_
         }
         __syncthreads();
 
-        if (!NV && p.do_row) {
+        if (p.do_row) {
             float sv[S];
 #pragma unroll
             for (int s = 0; s < S; ++s) sv[s] = srow[s * p.rps + rsw];
