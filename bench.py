@@ -592,7 +592,7 @@ def run_gpu_gemm(args, dist: Dist) -> dict | None:
     b = nv.quantize(w, flags=nv.ROWWISE)
     del x, w
     outs = [torch.empty((m, n), dtype=torch.float32, device=dev) for _ in range(2)]
-    ws = nv.new_gemm_workspace(dev)
+    ws = nv.new_gemm_workspace(m, n, k, dev)
 
     def step(i):
         nv.gemm_per_token(a["q_row"], a["sf_row"], a["amax_row"], b["q_row"], b["sf_row"], b["amax_row"],

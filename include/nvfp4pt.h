@@ -241,8 +241,10 @@ NVFP4PT_API nvfp4pt_status nvfp4pt_requantize_colwise(const uint8_t* q_row, cons
                                                       float* absmax_bufs, float decay, void* workspace,
                                                       cudaStream_t stream);
 
-/* Bytes of the workspace of nvfp4pt_gemm_per_token (its device error word). */
-NVFP4PT_API size_t nvfp4pt_gemm_workspace_bytes(void);
+/* Bytes of the workspace of nvfp4pt_gemm_per_token for an m x n x k product: the device
+ * error word, then both operands' block scales rearranged into the layout of the copy
+ * into tensor memory (about (m + n) * k / 16 bytes). */
+NVFP4PT_API size_t nvfp4pt_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
  * nvfp4pt_gemm_per_token -- the GEMM of two per-token NVFP4 operands, rescaled in its
@@ -263,8 +265,9 @@ NVFP4PT_API size_t nvfp4pt_gemm_workspace_bytes(void);
  *   qa, sfa, amax_a  uint8 [m, k/2] codes, uint8 [m, k/16] E4M3 scales, fp32 [m] amax
  *   qb, sfb, amax_b  uint8 [n, k/2], uint8 [n, k/16], fp32 [n]
  *   d                fp32 [m, n] row-major, written in full
- *   workspace        nvfp4pt_gemm_workspace_bytes() bytes; holds the error word that
+ *   workspace        nvfp4pt_gemm_workspace_bytes(m, n, k) bytes; holds the error word that
  *                    nvfp4pt_workspace_error reads (a wait inside the kernel that gave up)
+ *                    and, written by the call, the block scales in tensor-memory copy layout
  * Block scales must be non-negative finite E4M3 codes (0x00..0x7E), as the cast writes.
  * m and n are multiples of 16, k a multiple of 256 (a row of block scales is then a
  * whole number of 16-byte units, as the tensor-memory-access copies require), all at

@@ -81,7 +81,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4pt_requantize_workspace_bytes.argtypes = [I64, I64, I]
         L.nvfp4pt_requantize_colwise.argtypes = [P, P, P, I64, I64, P, I, P, P, P, P, F, P, P]
         L.nvfp4pt_quantize_grouped_opts.argtypes = [P, I64, I64, P, I, I, P, P, P, P, P, P, P, F, P, P, P]
-        L.nvfp4pt_gemm_workspace_bytes.argtypes = []
+        L.nvfp4pt_gemm_workspace_bytes.argtypes = [I64, I64, I64]
         L.nvfp4pt_gemm_per_token.argtypes = [P, P, P, I64, P, P, P, I64, I64, P, P, P]
         for name in EXPORTS[2:]:
             getattr(L, name).restype = I
@@ -270,8 +270,8 @@ def gemm_per_token(qa: torch.Tensor, sfa: torch.Tensor, amax_a: torch.Tensor, qb
     pab = _buf(amax_b, "amax_b", torch.float32, n, dev)
     out = torch.empty((m, n), dtype=torch.float32, device=qa.device) if out is None else out
     po = _buf(out, "out", torch.float32, m * n, dev)
-    ws = new_gemm_workspace(qa.device) if workspace is None else workspace
-    pw = _buf(ws, "workspace", torch.uint8, gemm_workspace_bytes(), dev)
+    ws = new_gemm_workspace(m, n, k, qa.device) if workspace is None else workspace
+    pw = _buf(ws, "workspace", torch.uint8, gemm_workspace_bytes(m, n, k), dev)
     _require_cuda(qa, "qa")
     st = lib().nvfp4pt_gemm_per_token(_ptr(qa), psa, paa, m, pqb, psb, pab, n, k, po, pw,
                                       _stream(stream, qa.device))
@@ -279,13 +279,13 @@ def gemm_per_token(qa: torch.Tensor, sfa: torch.Tensor, amax_a: torch.Tensor, qb
     return out
 
 
-@functools.lru_cache(maxsize=1)
-def gemm_workspace_bytes() -> int:
-    return int(lib().nvfp4pt_gemm_workspace_bytes())
+@functools.lru_cache(maxsize=256)
+def gemm_workspace_bytes(m: int, n: int, k: int) -> int:
+    return int(lib().nvfp4pt_gemm_workspace_bytes(m, n, k))
 
 
-def new_gemm_workspace(device=None) -> torch.Tensor:
-    return torch.empty(gemm_workspace_bytes(), dtype=torch.uint8, device=device)
+def new_gemm_workspace(m: int, n: int, k: int, device=None) -> torch.Tensor:
+    return torch.empty(gemm_workspace_bytes(m, n, k), dtype=torch.uint8, device=device)
 
 
 @functools.lru_cache(maxsize=256)

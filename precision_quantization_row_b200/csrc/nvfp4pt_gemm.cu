@@ -1,5 +1,6 @@
-// Host side of nvfp4pt_gemm_per_token (include/nvfp4pt.h): argument checks, the four
-// TMA descriptors of the operands and the launch of the tcgen05 kernel.
+// Host side of nvfp4pt_gemm_per_token (include/nvfp4pt.h): argument checks, the scale
+// rearrangement into the workspace, the TMA descriptors of the codes and the launch of
+// the tcgen05 kernel.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -69,11 +70,20 @@ nvfp4pt_status byte_map(CUtensorMap* map, const void* base, int64_t rows, int64_
     return r == CUDA_SUCCESS ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }
 
+int64_t align256(int64_t n) { return (n + 255) & ~int64_t(255); }
+
+// Workspace: the error word, then A's and B's block scales in copy layout (A's rows padded
+// to whole 128-row blocks, B's to whole 256-row tiles).
+int64_t sfa_pre_bytes(int64_t m, int64_t k) { return align256((m + kGemmBM - 1) / kGemmBM * kGemmBM * (k / 16)); }
+int64_t sfb_pre_bytes(int64_t n, int64_t k) { return align256((n + kGemmBN - 1) / kGemmBN * kGemmBN * (k / 16)); }
 }  // namespace
 
 extern "C" {
-
-size_t nvfp4pt_gemm_workspace_bytes(void) { return 256; }
+size_t nvfp4pt_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k)
+{
+    if (m < 0 || n < 0 || k < 0 || m > kMaxDim || n > kMaxDim || k > kMaxDim) return 256;
+    return (size_t)(256 + sfa_pre_bytes(m, k) + sfb_pre_bytes(n, k));
+}
 
 nvfp4pt_status nvfp4pt_gemm_per_token(const uint8_t* qa, const uint8_t* sfa, const float* amax_a, int64_t m,
                                       const uint8_t* qb, const uint8_t* sfb, const float* amax_b, int64_t n,
@@ -93,9 +103,7 @@ nvfp4pt_status nvfp4pt_gemm_per_token(const uint8_t* qa, const uint8_t* sfa, con
     GemmParams p;
     std::memset(&p, 0, sizeof p);
     if ((st = byte_map(&p.tmA, qa, m, k / 2, 128, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B)) != NVFP4PT_OK ||
-        (st = byte_map(&p.tmB, qb, n, k / 2, 128, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B)) != NVFP4PT_OK ||
-        (st = byte_map(&p.tmSfa, sfa, m, k / 16, 16, kGemmBM, CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4PT_OK ||
-        (st = byte_map(&p.tmSfb, sfb, n, k / 16, 16, kGemmBN, CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4PT_OK)
+        (st = byte_map(&p.tmB, qb, n, k / 2, 128, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B)) != NVFP4PT_OK)
         return st;
     p.m = m;
     p.n = n;
@@ -104,12 +112,24 @@ nvfp4pt_status nvfp4pt_gemm_per_token(const uint8_t* qa, const uint8_t* sfa, con
     p.amax_b = amax_b;
     p.d = d;
     p.err = static_cast<uint32_t*>(workspace);
+    uint8_t* sfa_pre = static_cast<uint8_t*>(workspace) + 256;
+    uint8_t* sfb_pre = sfa_pre + sfa_pre_bytes(m, k);
+    p.sfa_pre = sfa_pre;
+    p.sfb_pre = sfb_pre;
     if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess) return NVFP4PT_ERR_CUDA;
     p.m_tiles = (int32_t)((m + kGemmBM - 1) / kGemmBM);
     p.n_tiles = (int32_t)((n + kGemmBN - 1) / kGemmBN);
     const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
-    // one persistent CTA per SM (or per tile, when there are fewer tiles)
-    const int grid = (int)std::min<int64_t>(tiles, g_sms[dev_index()]);
+    const int sms = g_sms[dev_index()];
+    // the scales in copy layout, then one persistent CTA per SM (or per tile, when there
+    // are fewer tiles)
+    const int64_t ks = k / kGemmBK;
+    const int64_t ma = (int64_t)p.m_tiles * kGemmBM, nb = (int64_t)p.n_tiles * kGemmBN;
+    const int ga = (int)std::max<int64_t>(1, std::min<int64_t>((ma * ks + 255) / 256, 8 * (int64_t)sms));
+    const int gb = (int)std::max<int64_t>(1, std::min<int64_t>((nb * ks + 255) / 256, 8 * (int64_t)sms));
+    gemm_sf_prep<<<ga, 256, 0, stream>>>(sfa, m, ma, ks, sfa_pre);
+    gemm_sf_prep<<<gb, 256, 0, stream>>>(sfb, n, nb, ks, sfb_pre);
+    const int grid = (int)std::min<int64_t>(tiles, sms);
     gemm_per_token_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
 }

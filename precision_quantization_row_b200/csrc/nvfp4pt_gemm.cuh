@@ -9,13 +9,15 @@
 // (TransformerEngine PR #3045 "Add NVFP4 per-token quantization recipe": a GEMM that
 // rescales with the per-row and per-column outer-amax vectors inside its epilogue).
 //
-// A persistent CTA per SM takes 128 x 256 tiles of D in turn:
+// First gemm_sf_prep writes each operand's block scales into the workspace in the
+// layout of the scale copy into tensor memory (one contiguous 2048-byte piece per
+// 128-row block and 256-element K step). Then a persistent CTA per SM takes 128 x 256
+// tiles of D in turn:
 //   warp 0       TMA producer: per 256-element K step, the A and B code tiles (128-byte
-//                rows, 128-byte swizzle) and the A and B block-scale rows (16 bytes
-//                each), four stages deep, running ahead into the next tile.
-//   warp 1       allocates tensor memory; its lanes rearrange the block scales in place
-//                into the layout of the scale copy, and lane 0 issues the copies into
-//                tensor memory (tcgen05.cp) and the four block-scaled MMAs of the step
+//                rows, 128-byte swizzle) and the A and B scale pieces (bulk copies),
+//                four stages deep, running ahead into the next tile.
+//   warp 1       allocates tensor memory; lane 0 issues the scale copies into tensor
+//                memory (tcgen05.cp) and the four block-scaled MMAs of the step
 //                (tcgen05.mma kind::mxf4nvf4, 16-element E4M3 scale vectors).
 //   warps 2..9   epilogue: each drains 32 rows x 128 columns of the fp32 accumulator
 //                into registers (tcgen05.ld) and frees it, so the next tile's MMAs run
@@ -39,10 +41,11 @@ constexpr int kGemmTmemCols = 512;     // accumulator 256 columns + scale factor
 // shared memory of one stage (offsets from the 1024-aligned stage base)
 constexpr int kGsA = 0;                               // A codes  128 x 128 B
 constexpr int kGsB = kGsA + kGemmBM * 128;            // B codes  256 x 128 B
-constexpr int kGsSfa = kGsB + kGemmBN * 128;          // A scales 128 x 16 B, then in copy layout
-constexpr int kGsSfb = kGsSfa + kGemmBM * 16;         // B scales 256 x 16 B, then in copy layout
+constexpr int kGsSfa = kGsB + kGemmBN * 128;          // A scales: one 2048-byte piece in copy layout
+constexpr int kGsSfb = kGsSfa + kGemmBM * 16;         // B scales: two pieces
 constexpr int kGemmStageBytes = kGsSfb + kGemmBN * 16;
-constexpr int kGemmTxBytes = kGemmStageBytes;         // bytes the TMA brings per stage
+constexpr int kGemmTxBytes = kGemmStageBytes;         // bytes the copies bring per stage
+constexpr int kGemmSfPiece = 2048;                     // scales of 128 rows x one 256-element K step
 constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024;   // + room to align the stages to 1024
 
 // tensor memory columns (lane field 0)
@@ -53,9 +56,9 @@ constexpr uint32_t kTmSfb = 272;    // 8 per MMA K step: B row 32c + i of a step
 struct GemmParams {
     CUtensorMap tmA;     // codes of A: uint8 [M, K/2], box 128 x 128, 128-byte swizzle
     CUtensorMap tmB;     // codes of B: uint8 [N, K/2], box 128 x 256, 128-byte swizzle
-    CUtensorMap tmSfa;   // scales of A: uint8 [M, K/16], box 16 x 128
-    CUtensorMap tmSfb;   // scales of B: uint8 [N, K/16], box 16 x 256
     int64_t m, n, k;
+    const uint8_t* sfa_pre;   // A's scales in copy layout: [ceil(M/128)][K/256] pieces
+    const uint8_t* sfb_pre;   // B's scales in copy layout: [2 ceil(N/256)][K/256] pieces
     const float* amax_a;
     const float* amax_b;
     float* d;            // [M, N] fp32
@@ -152,35 +155,33 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[3
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void fence_proxy_async_smem()
+
+// One contiguous copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global into shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
 {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
-// A [128 * nblk][16 B] scale tile, rearranged in place into the copy layout: 128-row
-// block b becomes four 512-byte pieces at b * 2048 + kb * 512 (kb: the MMA K step),
-// whose 16-byte line i holds the kb-th scale word (4 scales) of the block's rows i,
-// i + 32, i + 64, i + 96. A block's pieces take exactly its own 2048 bytes, so the
-// warp reads a block whole before it writes it. Lane i of a warp.
-__device__ __forceinline__ void sf_to_copy_layout(uint32_t base, int lane, int nblk)
+// An operand's block scales ([rows, K/16]: 16 bytes per row and 256-element K step) in the
+// layout of tcgen05.cp.32x128b.warpx4: for each 128-row block and K step a 2048-byte piece
+// whose 512-byte part kb holds, in its 16-byte line i, the kb-th 4-byte scale word of the
+// block's rows i, i + 32, i + 64, i + 96. Rows from `rows` up to `padded_rows` get zero
+// scales. Thread u takes row u / ksteps, K step u % ksteps (the reads are contiguous).
+__global__ void __launch_bounds__(256) gemm_sf_prep(const uint8_t* sf, int64_t rows, int64_t padded_rows,
+                                                    int64_t ksteps, uint8_t* pre)
 {
-    for (int b = 0; b < nblk; ++b) {
-        const uint32_t blk = base + 2048u * (uint32_t)b;
-        uint4 r[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) r[c] = lds128(blk + 16u * (uint32_t)(32 * c + lane));
-        __syncwarp();
-        const uint32_t w0[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
-        const uint32_t w1[4] = {r[1].x, r[1].y, r[1].z, r[1].w};
-        const uint32_t w2[4] = {r[2].x, r[2].y, r[2].z, r[2].w};
-        const uint32_t w3[4] = {r[3].x, r[3].y, r[3].z, r[3].w};
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t a = blk + 512u * (uint32_t)kb + 16u * (uint32_t)lane;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0[kb]), "r"(w1[kb]),
-                         "r"(w2[kb]), "r"(w3[kb])
-                         : "memory");
-        }
+    const int64_t total = padded_rows * ksteps;
+    for (int64_t u = (int64_t)blockIdx.x * 256 + threadIdx.x; u < total; u += (int64_t)gridDim.x * 256) {
+        const int64_t r = u / ksteps, ks = u - r * ksteps;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < rows) v = __ldg(reinterpret_cast<const uint4*>(sf + r * (ksteps * 16) + ks * 16));
+        uint8_t* dst = pre + ((r >> 7) * ksteps + ks) * kGemmSfPiece + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+        *reinterpret_cast<uint32_t*>(dst) = v.x;
+        *reinterpret_cast<uint32_t*>(dst + 512) = v.y;
+        *reinterpret_cast<uint32_t*>(dst + 1024) = v.z;
+        *reinterpret_cast<uint32_t*>(dst + 1536) = v.w;
     }
 }
 
@@ -218,8 +219,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
         fence_mbar_init();
         prefetch_tensormap(&p.tmA);
         prefetch_tensormap(&p.tmB);
-        prefetch_tensormap(&p.tmSfa);
-        prefetch_tensormap(&p.tmSfb);
     }
     if (warp == 1) tmem_alloc(smem_u32(&tmem_slot_mem), kGemmTmemCols);
     tc_fence_before();
@@ -247,8 +246,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
                     mbar_arrive_expect_tx(fb, kGemmTxBytes);
                     tma_load_2d(st + kGsA, &p.tmA, ks * 128, m0, fb);
                     tma_load_2d(st + kGsB, &p.tmB, ks * 128, n0, fb);
-                    tma_load_2d(st + kGsSfa, &p.tmSfa, ks * 16, m0, fb);
-                    tma_load_2d(st + kGsSfb, &p.tmSfb, ks * 16, n0, fb);
+                    const int64_t pa = ((int64_t)(m0 / 128) * ksteps + ks) * kGemmSfPiece;
+                    bulk_load(st + kGsSfa, p.sfa_pre + pa, kGemmSfPiece, fb);
+                    for (int h = 0; h < kGemmBN / 128; ++h) {
+                        const int64_t pb = ((int64_t)(n0 / 128 + h) * ksteps + ks) * kGemmSfPiece;
+                        bulk_load(st + kGsSfb + kGemmSfPiece * h, p.sfb_pre + pb, kGemmSfPiece, fb);
+                    }
                 }
             }
             // copies must not land in freed shared memory: wait for the last ones issued
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ scale layout + MMA issue
+        // ------------------------------------------------------------ MMA issue
         const uint32_t idesc = gemm_idesc();
         int64_t it = 0;
         int j = 0;    // tiles of this CTA so far
@@ -281,10 +284,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
                     break;
                 }
                 const uint32_t st = smem0 + s * kGemmStageBytes;
-                sf_to_copy_layout(st + kGsSfa, lane, kGemmBM / 128);
-                sf_to_copy_layout(st + kGsSfb, lane, kGemmBN / 128);
-                fence_proxy_async_smem();
-                __syncwarp();
                 if (lane == 0) {
                     tc_fence_after();
 #pragma unroll

@@ -177,7 +177,10 @@ def test_gemm_rejections(L):
     g = lambda qa=None, m=128, n=256, k=512, d=None, ws=None, sfb=None: L.nvfp4pt_gemm_per_token(
         P() if qa is None else qa, P(), P(), m, P(), P() if sfb is None else sfb, P(), n, k,
         P() if d is None else d, P() if ws is None else ws, None)
-    assert L.nvfp4pt_gemm_workspace_bytes() >= 4
+    # the error word, then both operands' block scales (rows padded to 128 for A, 256 for B)
+    assert L.nvfp4pt_gemm_workspace_bytes(16, 16, 256) == 256 + 128 * 16 + 256 * 16
+    assert L.nvfp4pt_gemm_workspace_bytes(16384, 8192, 8192) == 256 + (16384 + 8192) * 512
+    assert L.nvfp4pt_gemm_workspace_bytes(-1, 16, 256) == 256
     assert L.nvfp4pt_gemm_per_token(None, P(), P(), 16, P(), P(), P(), 16, 256, P(), P(), None) == 1
     assert L.nvfp4pt_gemm_per_token(P(), P(), P(), 16, P(), P(), P(), 16, 256, None, P(), None) == 1
     assert L.nvfp4pt_gemm_per_token(P(), P(), P(), 16, P(), P(), P(), 16, 256, P(), None, None) == 1

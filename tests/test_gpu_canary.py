@@ -117,7 +117,7 @@ def test_gemm():
     aa = torch.rand(m, device="cuda", generator=g)
     ab = torch.rand(n, device="cuda", generator=g)
     d_raw, d = guarded((m, n), torch.float32, "cuda")
-    ws_raw, ws = guarded((nv.gemm_workspace_bytes(),), torch.uint8, "cuda")
+    ws_raw, ws = guarded((nv.gemm_workspace_bytes(m, n, k),), torch.uint8, "cuda")
     nv.gemm_per_token(qa, sfa, aa, qb, sfb, ab, out=d, workspace=ws)
     _check([d_raw, ws_raw], {"d": d}, {"d": nv.gemm_per_token(qa, sfa, aa, qb, sfb, ab)})
 

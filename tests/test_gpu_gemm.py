@@ -27,7 +27,7 @@ def _t(a):
 
 
 def gpu_gemm(qa, sfa, aa, qb, sfb, ab):
-    ws = nv.new_gemm_workspace("cuda")
+    ws = nv.new_gemm_workspace(qa.shape[0], qb.shape[0], 2 * qa.shape[1], "cuda")
     d = nv.gemm_per_token(_t(qa), _t(sfa), _t(aa), _t(qb), _t(sfb), _t(ab), workspace=ws)
     assert nv.workspace_error(ws) == 0
     return d.cpu().numpy().astype(np.float64)
@@ -124,7 +124,7 @@ def test_full_tiling_sampled(orc):
     sfb = torch.randint(0, 0x7F, (n, k // 16), dtype=torch.uint8, device="cuda", generator=g)
     aa = torch.rand(m, device="cuda", generator=g) * 10
     ab = torch.rand(n, device="cuda", generator=g) * 10
-    ws = nv.new_gemm_workspace("cuda")
+    ws = nv.new_gemm_workspace(m, n, k, "cuda")
     d = nv.gemm_per_token(qa, sfa, aa, qb, sfb, ab, workspace=ws)
     assert nv.workspace_error(ws) == 0
     rng = np.random.default_rng(9)
