@@ -64,30 +64,29 @@ __device__ __forceinline__ void rht16(float (&f)[16], uint32_t signs)
     for (int j = 0; j < 16; ++j) f[j] = __fmul_rn(f[j], 0.25f);
 }
 
-// Stochastic E2M1 code of y with the random word r (4 bits: sign in bit 3).
+// Stochastic E2M1 code of y with the random word r (4 bits: sign in bit 3), without
+// branches: for a = |y| < 6 the grid point lo at or below a, the gap to the next one and
+// lo's code come from a's bits --
+//   a >= 1 (biased exponent e = 127, 128, 129): lo = a with its significand cut to one
+//          bit, gap = 2^(e - 128), code 2 (e - 127) + 2 + (the significand's top bit);
+//   a < 1: lo = 0 or 0.5 (codes 0, 1), gap = 0.5 --
+// then f = (a - lo) / gap (exact: a - lo is exact and the gap a power of two) and the
+// code steps up iff r < ceil(f * 2^32).
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t r)
 {
-    const uint32_t sign = (__float_as_uint(y) >> 28) & 8u;
-    const float a = fabsf(y);
-    if (a >= 6.0f) return sign | 7u;
-    uint32_t c;
-    float lo, inv_gap;
-    if (a < 2.0f) {            // grid 0, 0.5, 1, 1.5: gap 0.5
-        c = __float2uint_rz(__fmul_rn(a, 2.0f));
-        lo = __fmul_rn((float)c, 0.5f);
-        inv_gap = 2.0f;
-    } else if (a < 4.0f) {     // grid 2, 3: gap 1
-        c = 4u + __float2uint_rz(__fsub_rn(a, 2.0f));
-        lo = (float)(c - 2u);
-        inv_gap = 1.0f;
-    } else {                   // 4 .. 6: gap 2
-        c = 6u;
-        lo = 4.0f;
-        inv_gap = 0.5f;
-    }
-    const float f = __fmul_rn(__fsub_rn(a, lo), inv_gap);           // exact
-    const uint32_t t = __float2uint_ru(__fmul_rn(f, 4294967296.0f));  // ceil(f * 2^32) < 2^32
-    return sign | (r < t ? c + 1u : c);
+    const uint32_t yb = __float_as_uint(y);
+    const uint32_t sign = (yb >> 28) & 8u;
+    const uint32_t ab = yb & 0x7FFFFFFFu;
+    const bool big = ab >= 0x3F800000u;                                  // a >= 1
+    const bool half = ab >= 0x3F000000u;                                 // a >= 0.5
+    const uint32_t lo_b = big ? (ab & 0xFFC00000u) : (half ? 0x3F000000u : 0u);
+    const uint32_t gap_b = big ? ((ab & 0x7F800000u) - 0x00800000u) : 0x3F000000u;
+    const uint32_t c = big ? 2u * ((ab >> 23) - 127u) + 2u + ((ab >> 22) & 1u) : (half ? 1u : 0u);
+    const float f = __fmul_rn(__fsub_rn(__uint_as_float(ab), __uint_as_float(lo_b)),
+                              __uint_as_float(0x7F000000u - gap_b));   // times 1 / gap
+    const uint32_t t = __float2uint_ru(__fmul_rn(f, 4294967296.0f));   // ceil(f * 2^32) < 2^32
+    const uint32_t code = ab >= 0x40C00000u ? 7u : (r < t ? c + 1u : c);   // a >= 6 saturates
+    return sign | code;
 }
 
 // The block steps with IEEE divisions (the block amax of transformed values is any
