@@ -224,6 +224,8 @@ def quantize_timed(x: torch.Tensor, events, flags: int = ROWWISE | COLWISE, absm
     pa = _opt_buf(absmax, "absmax", torch.float32, 1, dev)
     pw = _buf(ws, "workspace", torch.uint8, workspace_bytes(rows, cols, 1), dev)
     _require_cuda(x, "x")
+    if any(e.cuda_event == 0 for e in events):
+        raise ValueError("every event must have been recorded once (torch creates it lazily)")
     evs = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     st = lib().nvfp4pt_quantize_timed(_ptr(x), rows, cols, flags, *p, pa, ctypes.c_float(decay), pw,
                                       _stream(stream, x.device), evs)

@@ -565,9 +565,11 @@ nvfp4pt_status run_requant(const uint8_t* q, const uint8_t* sf, const float* ama
             encode_u8_map(&p.tm_sf, sf, rows, cols / 16, kRtCols / 16, kRtRows) != NVFP4PT_OK ||
             encode_f32_vector_map(&p.tm_amax, amax, rows, kRtRows) != NVFP4PT_OK)
             return NVFP4PT_ERR_CUDA;
-        const int grid = (int)std::min<int64_t>((cols / kRtCols) * tsteps, 2 * sms);
-        if (launch(rq_tile<MAXG, false>, grid, kSmemRqTile, stream, p, true, kRtThreads) != cudaSuccess ||
-            launch(rq_tile<MAXG, true>, grid, kSmemRqTile, stream, p, true, kRtThreads) != cudaSuccess)
+        const int64_t units = (cols / kRtCols) * tsteps;
+        const int grid1 = (int)std::min<int64_t>(units, kRtCtasMax * sms);
+        const int grid2 = (int)std::min<int64_t>(units, kRtCtasEnc * sms);
+        if (launch(rq_tile<MAXG, false>, grid1, kSmemRqTileMax, stream, p, true, kRtThreads) != cudaSuccess ||
+            launch(rq_tile<MAXG, true>, grid2, kSmemRqTile, stream, p, true, kRtThreads) != cudaSuccess)
             return NVFP4PT_ERR_CUDA;
         return NVFP4PT_OK;
     }

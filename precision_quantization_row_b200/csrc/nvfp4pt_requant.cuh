@@ -420,15 +420,18 @@ __global__ void __launch_bounds__(kRqThreads, 2) rq_colenc(const __grid_constant
 // Both requantization passes again for rows a multiple of 256 wide (each row's scales
 // are then whole 16-byte pieces, as TMA needs): a CTA walks tiles of 256 columns x 64
 // rows down the matrix, TMA copies stay kRtStages tiles ahead of the warps (the codes,
-// the scales and the 64 rows' amaxes), and the warps read shared memory only. Warp w
-// takes the 16-row block w & 3 of a tile and its 128-column half w >> 2; lane l takes
-// columns 4l .. 4l+3 of that half over all 16 rows, so every lane holds whole 16-row
-// column blocks. ENC = false keeps column maxima (rq_colmax's job); ENC = true encodes
-// (rq_colenc's job): the warps leave their lanes' 8-byte column segments and scale bytes
-// in a staging tile and, after the CTA's barrier, each thread writes one column's 32
-// code bytes and 4 scale bytes. Units are (256-column chunk, 64-row step) pairs in
+// the scales and the 64 rows' amaxes), and the warps read shared memory only; each lane
+// decodes whole 32-bit words of codes (eight elements of one block of its row).
+// ENC = false keeps column maxima (rq_colmax's job): warp w takes rows 8w .. 8w+7 of a
+// tile and lane l columns 8l .. 8l+7. ENC = true encodes (rq_colenc's job): warp w takes
+// the 16-row block w & 3 and the 128-column half w >> 2, and lanes l and l + 16 take the
+// half's columns 8l .. 8l+7, rows 0-7 and 8-15 of the block; the pair joins its block
+// maxima by one shuffle, each lane finds the block scales of four of the columns, and the
+// pair swaps codes so that each lane leaves four whole 8-byte column segments and their
+// scale bytes in a staging tile. After the CTA's barrier each thread writes one column's
+// 32 code bytes and 4 scale bytes. Units are (256-column chunk, 64-row step) pairs in
 // chunk-major order, the steps of each token group starting at its first row; each CTA
-// takes a contiguous run.
+// takes a contiguous run and walks it with a cursor.
 constexpr int kRtThreads = 256;
 constexpr int kRtCols = 256;
 constexpr int kRtRows = 64;
@@ -438,7 +441,10 @@ constexpr int kRtScaleBytes = kRtRows * kRtCols / 16;                         //
 constexpr int kRtStageBytes = kRtCodeBytes + kRtScaleBytes + kRtRows * 4;    // + the amaxes: 9472
 constexpr int kRtOutCodes = 4 * kRtCols * 8;                                  // [row block][column] 8 bytes
 constexpr int kRtOutBytes = kRtOutCodes + 4 * kRtCols;                        // + [row block][column] scale bytes
-constexpr int kSmemRqTile = kRtStages * kRtStageBytes + 2 * kRtOutBytes + 128;
+constexpr int kSmemRqTile = kRtStages * kRtStageBytes + 2 * kRtOutBytes + 128;   // ENC
+constexpr int kSmemRqTileMax = kRtStages * kRtStageBytes + 128;                  // !ENC: no staging
+constexpr int kRtCtasMax = 4;   // !ENC CTAs per SM (56 registers, 38 KB)
+constexpr int kRtCtasEnc = 2;   // ENC CTAs per SM (about 100 registers)
 
 struct RtUnit {
     int64_t chunk;
@@ -448,26 +454,51 @@ struct RtUnit {
     bool first;       // the group's first step
 };
 
+// A CTA's units are consecutive: a cursor walks them without a division per unit.
+struct RtCursor {
+    int64_t chunk;
+    int64_t k;   // step within the chunk
+    int g;       // the group holding step k (empty groups skipped)
+};
+
 template <int MAXG>
-__device__ __forceinline__ RtUnit rt_unit(const RqParams<MAXG>& p, int64_t u, int64_t steps)
+__device__ __forceinline__ void rt_seek(const RqParams<MAXG>& p, int64_t u, int64_t steps, RtCursor& c)
 {
-    RtUnit t;
-    t.chunk = u / steps;
-    const int64_t k = u - t.chunk * steps;
-    int g = 0;
+    c.chunk = u / steps;
+    c.k = u - c.chunk * steps;
+    c.g = 0;
     if (MAXG > 1) {
         int lo = 0, hi = p.num_groups;   // the last group whose first step is <= k
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (p.tstep_off[mid] <= k) lo = mid; else hi = mid;
+            if (p.tstep_off[mid] <= c.k) lo = mid; else hi = mid;
         }
-        g = lo;
+        c.g = lo;
     }
-    t.g = g;
-    t.row0 = p.row_off[g] + (k - p.tstep_off[g]) * kRtRows;
-    const int64_t left = p.row_off[g + 1] - t.row0;
+}
+
+template <int MAXG>
+__device__ __forceinline__ void rt_next(const RqParams<MAXG>& p, int64_t steps, RtCursor& c)
+{
+    if (++c.k == steps) {
+        c.k = 0;
+        ++c.chunk;
+        c.g = 0;
+    }
+    if (MAXG > 1)
+        while (c.g + 1 < p.num_groups && p.tstep_off[c.g + 1] <= c.k) ++c.g;
+}
+
+template <int MAXG>
+__device__ __forceinline__ RtUnit rt_unit(const RqParams<MAXG>& p, const RtCursor& c)
+{
+    RtUnit t;
+    t.chunk = c.chunk;
+    t.g = c.g;
+    t.row0 = p.row_off[c.g] + (c.k - p.tstep_off[c.g]) * kRtRows;
+    const int64_t left = p.row_off[c.g + 1] - t.row0;
     t.nrows = left < kRtRows ? (int32_t)left : kRtRows;
-    t.first = k == p.tstep_off[g];
+    t.first = c.k == p.tstep_off[c.g];
     return t;
 }
 
@@ -503,7 +534,7 @@ __device__ __forceinline__ void rq_dequant4(uint32_t codes, uint32_t s2, float m
 }
 
 template <int MAXG, bool ENC>
-__global__ void __launch_bounds__(kRtThreads, 2) rq_tile(const __grid_constant__ RqParams<MAXG> p)
+__global__ void __launch_bounds__(kRtThreads, ENC ? kRtCtasEnc : kRtCtasMax) rq_tile(const __grid_constant__ RqParams<MAXG> p)
 {
     // The kernel after this one may launch early: it waits for this grid itself.
     griddep_launch_dependents();
@@ -536,8 +567,11 @@ __global__ void __launch_bounds__(kRtThreads, 2) rq_tile(const __grid_constant__
         prefetch_tensormap(&p.tm_amax);
     }
     __syncthreads();
-    auto issue = [&](int64_t i) {   // unit u0 + i into stage i % kRtStages (thread 0)
-        const RtUnit t = rt_unit(p, u0 + i, steps);
+    RtCursor pc;   // thread 0: the next unit to copy
+    if (tid == 0 && n > 0) rt_seek(p, u0, steps, pc);
+    auto issue = [&](int64_t i) {   // unit u0 + i (the cursor's) into stage i % kRtStages (thread 0)
+        const RtUnit t = rt_unit(p, pc);
+        rt_next(p, steps, pc);
         const int s = (int)(i % kRtStages);
         const uint32_t bar = bar0 + 8 * s, dst = stage0 + s * kRtStageBytes;
         mbar_arrive_expect_tx(bar, kRtStageBytes);
@@ -559,39 +593,48 @@ __global__ void __launch_bounds__(kRtThreads, 2) rq_tile(const __grid_constant__
     }
     if (n <= 0) return;   // no barrier follows for a CTA without units
 
-    const int cl = half * 128 + 4 * lane;   // this lane's first column in the chunk
-    uint32_t acc0 = 0u, acc1 = 0u;          // !ENC: column maxima since the last flush
+    // !ENC: warp w takes rows 8w .. 8w+7 of the step, lane l columns 8l .. 8l+7 of the chunk.
+    // ENC: warp (rb, half) takes the 16-row block rb and the 128-column half; lanes l and
+    // l + 16 share columns half*128 + 8(l & 15) .. +7, rows 0-7 and 8-15 of the block.
+    const int pl = lane & 15;
+    const int sub = lane >> 4;
+    const int cl = ENC ? half * 128 + 8 * pl : 8 * lane;   // this lane's first column in the chunk
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};     // !ENC: column maxima since the last flush
     int64_t acc_chunk = -1;
     int acc_g = -1;
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};     // ENC: outer scales of the lane's columns
+    float sc[8];                            // ENC: outer scales of the lane's columns
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sc[j] = 0.f;
     int64_t sc_chunk = -1;
     int sc_g = -1;
 
     // !ENC: raise colmax and obs with the maxima kept since the last flush
     auto flush = [&]() {
         if (acc_chunk < 0) return;
-        acc0 &= 0x7FFF7FFFu;
-        acc1 &= 0x7FFF7FFFu;
-        // lanes 2k and 2k+1 hold 8 contiguous columns: the even one raises all 8
-        const uint32_t n0 = __shfl_down_sync(0xFFFFFFFFu, acc0, 1);
-        const uint32_t n1 = __shfl_down_sync(0xFFFFFFFFu, acc1, 1);
-        if ((lane & 1) == 0 && (acc0 | acc1 | n0 | n1))
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] &= 0x7FFF7FFFu;
+        if (acc[0] | acc[1] | acc[2] | acc[3])
             red_max_bf16x8(reinterpret_cast<uint32_t*>(p.colmax + (int64_t)acc_g * cols + acc_chunk * kRtCols + cl),
-                           acc0, acc1, n0, n1);
+                           acc[0], acc[1], acc[2], acc[3]);
         if (p.obs) {
-            uint32_t mx = max(max(acc0 & 0xFFFFu, acc0 >> 16), max(acc1 & 0xFFFFu, acc1 >> 16));
+            uint32_t mx = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mx = max(mx, max(acc[j] & 0xFFFFu, acc[j] >> 16));
             mx = __reduce_max_sync(0xFFFFFFFFu, mx << 16);
             if (lane == 0 && mx) red_max_f32(p.obs + acc_g, mx);
         }
-        acc0 = acc1 = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = 0u;
     };
 
-    for (int64_t i = 0; i < n; ++i) {
+    RtCursor cc;
+    rt_seek(p, u0, steps, cc);
+    for (int64_t i = 0; i < n; ++i, rt_next(p, steps, cc)) {
         const int s = (int)(i % kRtStages);
-        const RtUnit t = rt_unit(p, u0 + i, steps);
+        const RtUnit t = rt_unit(p, cc);
         const bool ok = mbar_wait_bounded(bar0 + 8 * s, (uint32_t)((i / kRtStages) & 1));
         const uint8_t* st = smem + s * kRtStageBytes;
-        const bool rok = ok && 16 * rb < t.nrows;
+        const bool rok = ok && (ENC ? 16 * rb : 8 * warp) < t.nrows;
         uint8_t* os = ostage + (i & 1) * kRtOutBytes;
 
         if (!ENC && (t.chunk != acc_chunk || t.g != acc_g)) {
@@ -600,74 +643,94 @@ __global__ void __launch_bounds__(kRtThreads, 2) rq_tile(const __grid_constant__
             acc_g = t.g;
         }
         if (ENC && (t.chunk != sc_chunk || t.g != sc_g)) {
-            // outer scales of the lane's four columns, from the group's column maxima
+            // outer scales of the lane's eight columns, from the group's column maxima
             sc_chunk = t.chunk;
             sc_g = t.g;
             const int64_t c = t.chunk * kRtCols + cl;
-            const uint2 a = *reinterpret_cast<const uint2*>(p.colmax + (int64_t)t.g * cols + c);
-            const float a4[4] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y)};
+            const uint4 a = *reinterpret_cast<const uint4*>(p.colmax + (int64_t)t.g * cols + c);
+            const float a8[8] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
+                                 bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w)};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sc[j] = s_enc_of(a4[j]);
-            if (t.first && rb == 0)
-                *reinterpret_cast<float4*>(p.amax_col + (int64_t)t.g * cols + c) =
-                    make_float4(a4[0], a4[1], a4[2], a4[3]);
+            for (int j = 0; j < 8; ++j) sc[j] = s_enc_of(a8[j]);
+            if (t.first && rb == 0 && sub == 0) {
+                float4* d = reinterpret_cast<float4*>(p.amax_col + (int64_t)t.g * cols + c);
+                d[0] = make_float4(a8[0], a8[1], a8[2], a8[3]);
+                d[1] = make_float4(a8[4], a8[5], a8[6], a8[7]);
+            }
         }
 
         if (rok) {
-            // decode scales of the warp's 16 rows: lane r finds row r's, the warp shares them
             const float* amax_st = reinterpret_cast<const float*>(st + kRtCodeBytes + kRtScaleBytes);
-            const float dl = __fdiv_rn(amax_st[16 * rb + (lane & 15)], 2688.0f);
-            const uint8_t* cq = st + (16 * rb) * (kRtCols / 2) + half * 64 + 2 * lane;
-            const uint8_t* cs = st + kRtCodeBytes + (16 * rb) * (kRtCols / 16) + half * 8 + (lane >> 2);
-            uint32_t x[16][2];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                // the lane's two code bytes, taken from the aligned 32-bit word and moved to
-                // the low half (fed from a 16-bit load, the byte split below read wrong bytes)
-                const uint32_t w32 = *reinterpret_cast<const uint32_t*>(cq - 2 * (lane & 1) + r * (kRtCols / 2));
-                const uint32_t codes = __byte_perm(w32, 0u, (lane & 1) ? 0x4432u : 0x4410u);
-                const uint32_t sfc = cs[r * (kRtCols / 16)];
-                uint32_t s2;
-                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"((uint16_t)(sfc * 0x0101u)));
-                rq_dequant4(codes, s2, __shfl_sync(0xFFFFFFFFu, dl, r), x[r][0], x[r][1]);
-            }
-
             if (!ENC) {
+                // decode scales of the warp's 8 rows: lane r finds row r's, the warp shares them
+                const float dl = __fdiv_rn(amax_st[8 * warp + (lane & 7)], 2688.0f);
+                const uint8_t* cq = st + (8 * warp) * (kRtCols / 2) + 4 * lane;
+                const uint8_t* cs = st + kRtCodeBytes + (8 * warp) * (kRtCols / 16) + (lane >> 1);
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    acc0 = absmax2(acc0, x[r][0]);
-                    acc1 = absmax2(acc1, x[r][1]);
+                for (int r = 0; r < 8; ++r) {
+                    const uint32_t codes = *reinterpret_cast<const uint32_t*>(cq + r * (kRtCols / 2));
+                    uint32_t x[4];
+                    rq_dequant8(codes, cs[r * (kRtCols / 16)], __shfl_sync(0xFFFFFFFFu, dl, r), x);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[j] = absmax2(acc[j], x[j]);
                 }
             } else {
-                uint32_t bm[2];
+                // decode scales of the block's 16 rows: lanes r and r + 16 find row r's
+                const float dl = __fdiv_rn(amax_st[16 * rb + pl], 2688.0f);
+                const int r0 = 16 * rb + 8 * sub;   // the lane's first row in the step
+                const uint8_t* cq = st + r0 * (kRtCols / 2) + half * 64 + 4 * pl;
+                const uint8_t* cs = st + kRtCodeBytes + r0 * (kRtCols / 16) + half * 8 + (pl >> 1);
+                uint32_t x[8][4];   // the lane's row r: columns 2j, 2j+1 in word j
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    uint32_t m8[8];
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) m8[r] = absmax2(x[r][j], x[r + 8][j]);
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) m8[r] = absmax2(m8[r], m8[r + 4]);
-                    bm[j] = absmax2(absmax2(m8[0], m8[2]), absmax2(m8[1], m8[3])) & 0x7FFF7FFFu;
+                for (int r = 0; r < 8; ++r) {
+                    const uint32_t codes = *reinterpret_cast<const uint32_t*>(cq + r * (kRtCols / 2));
+                    rq_dequant8(codes, cs[r * (kRtCols / 16)], __shfl_sync(0xFFFFFFFFu, dl, 8 * sub + r), x[r]);
                 }
+                // block maxima of the eight columns over the block's 16 rows (both lanes)
+                uint32_t bm[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t m = absmax2(absmax2(absmax2(x[0][j], x[1][j]), absmax2(x[2][j], x[3][j])),
+                                               absmax2(absmax2(x[4][j], x[5][j]), absmax2(x[6][j], x[7][j])));
+                    bm[j] = absmax2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16)) & 0x7FFF7FFFu;
+                }
+                // each lane of the pair finds the scales of four columns (4 * sub ..), and
+                // the pair swaps the encode scales
+                const uint32_t ba = sub ? bm[2] : bm[0], bb = sub ? bm[3] : bm[1];
                 uint32_t sf01, sf23;
-                float e[4];
-                block_pair_scales_x2(bf16_lo(bm[0]), bf16_hi(bm[0]), sc[0], sc[1], sf01, e[0], e[1], rcp_tab);
-                block_pair_scales_x2(bf16_lo(bm[1]), bf16_hi(bm[1]), sc[2], sc[3], sf23, e[2], e[3], rcp_tab);
-                uint32_t q[8];   // column j: rows 0-7 in q[2j], rows 8-15 in q[2j+1]
+                float eo[4];
+                block_pair_scales_x2(bf16_lo(ba), bf16_hi(ba), sub ? sc[4] : sc[0], sub ? sc[5] : sc[1], sf01, eo[0],
+                                     eo[1], rcp_tab);
+                block_pair_scales_x2(bf16_lo(bb), bf16_hi(bb), sub ? sc[6] : sc[2], sub ? sc[7] : sc[3], sf23, eo[2],
+                                     eo[3], rcp_tab);
+                float e[8];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint32_t lo8[8] = {x[0][j], x[1][j], x[2][j], x[3][j], x[4][j], x[5][j], x[6][j], x[7][j]};
-                    const uint32_t hi8[8] = {x[8][j], x[9][j], x[10][j], x[11][j],
-                                             x[12][j], x[13][j], x[14][j], x[15][j]};
-                    q[4 * j] = encode8_col<false>(lo8, e[2 * j]);
-                    q[4 * j + 1] = encode8_col<false>(hi8, e[2 * j]);
-                    q[4 * j + 2] = encode8_col<true>(lo8, e[2 * j + 1]);
-                    q[4 * j + 3] = encode8_col<true>(hi8, e[2 * j + 1]);
+                for (int k = 0; k < 4; ++k) {
+                    const float ep = __shfl_xor_sync(0xFFFFFFFFu, eo[k], 16);
+                    e[k] = sub ? ep : eo[k];
+                    e[4 + k] = sub ? eo[k] : ep;
                 }
-                uint4* oc = reinterpret_cast<uint4*>(os + rb * (kRtCols * 8) + cl * 8);
-                oc[0] = make_uint4(q[0], q[1], q[2], q[3]);
-                oc[1] = make_uint4(q[4], q[5], q[6], q[7]);
-                *reinterpret_cast<uint32_t*>(os + kRtOutCodes + rb * kRtCols + cl) = sf01 | (sf23 << 16);
+                uint32_t q[8];   // column k of the lane's eight: the codes of the lane's eight rows
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t c8[8] = {x[0][j], x[1][j], x[2][j], x[3][j], x[4][j], x[5][j], x[6][j], x[7][j]};
+                    q[2 * j] = encode8_col<false>(c8, e[2 * j]);
+                    q[2 * j + 1] = encode8_col<true>(c8, e[2 * j + 1]);
+                }
+                // the lane stages columns 4 * sub .. 4 * sub + 3 whole: rows 0-7 and 8-15
+                uint32_t lo[4], hi[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t keep = sub ? q[4 + k] : q[k];
+                    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, sub ? q[k] : q[4 + k], 16);
+                    lo[k] = sub ? recv : keep;
+                    hi[k] = sub ? keep : recv;
+                }
+                const int oc0 = cl + 4 * sub;
+                uint4* oc = reinterpret_cast<uint4*>(os + rb * (kRtCols * 8) + oc0 * 8);
+                oc[0] = make_uint4(lo[0], hi[0], lo[1], hi[1]);
+                oc[1] = make_uint4(lo[2], hi[2], lo[3], hi[3]);
+                *reinterpret_cast<uint32_t*>(os + kRtOutCodes + rb * kRtCols + oc0) = sf01 | (sf23 << 16);
             }
         }
 
