@@ -64,7 +64,7 @@ struct GemmParams {
     float* d;            // [M, N] fp32
     uint32_t* err;
     int32_t m_tiles;     // tiles along M
-    int32_t n_tiles;     // tiles along N; tile t is (t / n_tiles, t % n_tiles), CTA c takes c, c + grid, ...
+    int32_t n_tiles;     // tiles along N; tile t as gemm_tile maps it, CTA c takes c, c + grid, ...
 };
 
 // Block-scaled MMA instruction descriptor: E2M1 A and B (K-major), E4M3 scales, fp32
@@ -190,6 +190,21 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Tile t -> its first row of A and of B: groups of kGemmGroupM row blocks are walked
+// column-major (all tiles of the group's first column of B, then the next), so that the
+// CTAs running at one time share few slices of A and B.
+constexpr int kGemmGroupM = 8;
+__device__ __forceinline__ void gemm_tile(int64_t t, int32_t m_tiles, int32_t n_tiles, int32_t& m0, int32_t& n0)
+{
+    const int64_t per = (int64_t)kGemmGroupM * n_tiles;
+    const int64_t g = t / per;
+    const int64_t first = g * kGemmGroupM;
+    const int64_t gm = m_tiles - first < kGemmGroupM ? m_tiles - first : kGemmGroupM;
+    const int64_t r = t - g * per;
+    m0 = (int32_t)((first + r % gm) * kGemmBM);
+    n0 = (int32_t)((r / gm) * kGemmBN);
+}
+
 __device__ __forceinline__ void gemm_fail(uint32_t* err, uint32_t code)
 {
     atomicOr(err, code);
@@ -232,7 +247,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
             int64_t it = 0;   // K steps issued over all tiles
             bool ok = true;
             for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int32_t m0 = (int32_t)(t / p.n_tiles) * kGemmBM, n0 = (int32_t)(t % p.n_tiles) * kGemmBN;
+                int32_t m0, n0;
+                gemm_tile(t, p.m_tiles, p.n_tiles, m0, n0);
                 for (int ks = 0; ks < ksteps; ++ks, ++it) {
                     const int s = (int)(it % kGemmStages);
                     const uint32_t ph = (uint32_t)((it / kGemmStages) & 1);
@@ -314,7 +330,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_per_token_kernel(const _
         const int half = (warp - 2) >> 2;        // and its 128 columns of the tile
         int j = 0;
         for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
-            const int64_t m0 = (t / p.n_tiles) * kGemmBM, n0 = (t % p.n_tiles) * kGemmBN + 128 * half;
+            int32_t tm0, tn0;
+            gemm_tile(t, p.m_tiles, p.n_tiles, tm0, tn0);
+            const int64_t m0 = tm0, n0 = (int64_t)tn0 + 128 * half;
             const int64_t row = m0 + 32 * q + lane;
             // the column decode scales S_dec(b_n) of this warp's 128 columns, 4 per lane
             float sdec[4];
