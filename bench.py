@@ -694,7 +694,8 @@ def run_gpu_config(args, dist: Dist, config: str) -> dict | None:
         def step(i):
             outs[i % copies] = nv.quantize_weight_2d(xs[i % copies], out=outs[i % copies], workspace=ws,
                                                      stream=stream)
-        byts = 2 * (2 * m * k) + m * k // 2 + m * k // 16 + 4 * m   # read twice, rowwise out
+        # the weight once (a band's second read comes from L2), rowwise outputs
+        byts = 2 * m * k + m * k // 2 + m * k // 16 + 4 * m
     if config == "calib":
         args.steps = copies   # one step per activation of the stream
     secs, all_secs, clocks = timed_regions(args, dist, dev, stream, step)

@@ -19,7 +19,8 @@ DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("nvfp4pt_device.cuh", "nvfp4pt
                                                   "nvfp4pt_rowpass.cuh", "nvfp4pt_colpass.cuh",
                                                   "nvfp4pt_dequant.cuh", "nvfp4pt_internal.h",
                                                   "nvfp4pt_gemm.cuh", "nvfp4pt_xform.cuh",
-                                                  "nvfp4pt_requant.cuh", "nvfp4pt_colpass_tma.cuh")] + \
+                                                  "nvfp4pt_requant.cuh", "nvfp4pt_colpass_tma.cuh",
+                                                  "nvfp4pt_w2d.cuh")] + \
     [os.path.join(INCLUDE, f) for f in ("nvfp4pt.h", "nvfp4pt_timing.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

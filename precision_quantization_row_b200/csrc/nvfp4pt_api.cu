@@ -14,6 +14,7 @@
 #include "nvfp4pt_internal.h"
 #include "nvfp4pt_kernels.cuh"
 #include "nvfp4pt_rowpass.cuh"
+#include "nvfp4pt_w2d.cuh"
 #include "nvfp4pt_colpass.cuh"
 #include "nvfp4pt_colpass_tma.cuh"
 #include "nvfp4pt_dequant.cuh"
@@ -734,6 +735,24 @@ nvfp4pt_status nvfp4pt_quantize_weight_2d(const void* w, int64_t rows, int64_t c
     if (!aligned16(w) || !aligned16(static_cast<uint8_t*>(workspace)) || !aligned16(q_row) || !aligned16(sf_row) ||
         !aligned16(amax_row))
         return NVFP4PT_ERR_ALIGN;
+    if (cols <= 16 * kW2dMaxThreads) {
+        // one sweep: a CTA per 16-row band at a time, a thread per 16-column block
+        DeviceState* dev = nullptr;
+        if ((st = device_state(&dev)) != NVFP4PT_OK) return st;
+        W2dParams p;
+        std::memset(&p, 0, sizeof p);
+        p.w = static_cast<const uint16_t*>(w);
+        p.bands = rows / kW2dRows;
+        p.cols = cols;
+        p.nbc = (int32_t)(cols / 16);
+        p.amax_row = amax_row;
+        p.q_row = q_row;
+        p.sf_row = sf_row;
+        p.err = ws_err(workspace);
+        const int threads = std::min(kW2dMaxThreads, (p.nbc + 31) / 32 * 32);
+        const int grid = (int)std::min<int64_t>(p.bands, (int64_t)dev->sm_count * (kW2dMaxThreads / threads));
+        return launch(w2d_band, grid, 0, stream, p, true, threads) == cudaSuccess ? NVFP4PT_OK : NVFP4PT_ERR_CUDA;
+    }
     const int64_t off[2] = {0, rows};
     return run_cast<1>(w, rows, cols, off, 1, NVFP4PT_ROWWISE, q_row, sf_row, amax_row, nullptr, nullptr, nullptr,
                        nullptr, 0.0f, true, workspace, stream);
