@@ -267,3 +267,15 @@ def test_weight_2d(orc, shape):
     w = inputs.random_shape(17, *shape, "wide")
     got = to_np(nv.quantize_weight_2d(w.cuda()))
     compare(got, orc.quantize_weight_2d(w), label=f"w2d {shape}")
+
+
+@pytest.mark.parametrize("shape,kind", [((32, 8192), "wide"), ((48, 8208), "wide"), ((64, 4096), "zeros"),
+                                        ((32, 2048), "signed_zero"), ((48, 1024), "tiny"), ((16, 8192), "normal")],
+                         ids=lambda v: v if isinstance(v, str) else f"{v[0]}x{v[1]}")
+def test_weight_2d_band_edges(orc, shape, kind):
+    """The one-sweep weight cast at its edges: bands of 512 blocks (every thread of the
+    CTA holds one), the first width past it (8208: the two-kernel tile path), all-zero and
+    signed-zero weights and tiny magnitudes."""
+    w = inputs.random_shape(18, *shape, kind)
+    got = to_np(nv.quantize_weight_2d(w.cuda()))
+    compare(got, orc.quantize_weight_2d(w), label=f"w2d {shape} {kind}")
